@@ -1,0 +1,485 @@
+// Stage 2: exact sparse attention over the kept key blocks with mean correction for the
+// pruned ones (FlashPrefill V2 paper page, Figure 3: the exact and mean-correction streams
+// "merge inside the online softmax"; Figure 4: a pruned block J contributes
+// |B_J| e^{s_J} (vbar_J, 1); Table 7: CSR per KV head, PackGQA).
+//
+// One CTA owns one (sequence r, query block i, KV head g, part) work item.  Its rows are
+// the G query heads of group g packed against their shared KV head (PackGQA): an M tile is
+// 128 rows = (128 / B) heads x B tokens, and a CTA carries NT <= 2 M tiles that share every
+// K/V tile it loads.  The key stream of the row is
+//     [virtual tiles][kept blocks in ascending order]
+// where virtual tile v holds the pooled kbar/vbar of blocks [vB, vB + B): every pruned
+// block j < i enters there as one extra "key" with logit q.kbar_j*scale + ln n_j, so the
+// correction shares the exact path's MMAs and online softmax; kept blocks and blocks >= i
+// are masked out of the virtual tiles.  The last kept block is the diagonal (causal mask).
+//
+// Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S,
+//                    mask, online max with lazy O rescale (only when the running max grows
+//                    by more than 2^8), write P (bf16 / e4m3 / f32) back over S in TMEM,
+//                    and finally normalise O and store it.
+//   warp 8           producer: builds the kept-block bitmask, issues TMA loads of Q once and
+//                    of K/V (or kbar/vbar) tiles into an NSLOT ring of shared-memory slots.
+//   warp 9           MMA issuer (one thread): S_s = Q_s K^T (SS form) and O_s += P_s V (A
+//                    operand P read from TMEM), tcgen05.commit to mbarriers.
+// TMEM: S0 | S1 | O0 | O1 (512 columns); P_s aliases S_s.
+#include <math_constants.h>
+
+#include "fp2_device.cuh"
+#include "fp2_kernels.h"
+
+namespace fp2 {
+
+template <int DT, int D, int BN>
+struct AttnCfg {
+  static constexpr int ELT = DT == 0 ? 4 : (DT == 1 ? 2 : 1);
+  static constexpr int KIND = DT == 0 ? 0 : (DT == 1 ? 1 : 2);
+  static constexpr uint32_t FMT = DT == 0 ? 2u : (DT == 1 ? 1u : 0u);  // tf32 / bf16 / e4m3
+  static constexpr int KCH = 128 / ELT;  // elements in one 128-byte swizzled row
+  static constexpr int DCH = D / KCH;    // 128-byte chunks along d
+  static constexpr int UK = 32 / ELT;    // K extent of one MMA instruction (32 bytes)
+  static constexpr int BM = 128;
+  static constexpr int Q_BYTES = BM * D * ELT;
+  static constexpr int KV_BYTES = BN * D * ELT;
+  static constexpr int TILE_BUDGET = 200 * 1024;
+  static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES) / KV_BYTES;
+  static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
+  static constexpr int S_COL0 = 0, S_COL1 = BN;
+  static constexpr int O_COL0 = 2 * BN, O_COL1 = 2 * BN + D;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_S = make_idesc(FMT, FMT, 0, 0, 128, BN);
+  static constexpr uint32_t IDESC_PV = make_idesc(FMT, FMT, 0, 1, 128, D);
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_MASK = OFF_MISC + 16;
+  // At least 116 KB so that a second CTA never shares the SM (each CTA holds all 512 TMEM columns).
+  static constexpr int SMEM_RAW = OFF_MASK + FP2_MAX_BLOCKS / 8 + 1024;
+  static constexpr int SMEM_BYTES = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
+  static_assert(NSLOT >= 2, "K/V ring needs at least two slots");
+  static_assert(2 * BN + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(D % KCH == 0 && BN % UK == 0 && D % 32 == 0 && BN % 32 == 0, "tile shape");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+};
+
+// tcgen05.ld of 32 columns followed by its wait, in one statement so that no use of the
+// registers can be scheduled before the data has landed.
+FP2_DEVICE void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Bit e of the result is set when pooled block (base + e) is a pruned block of query block i:
+// strictly left of the diagonal and absent from the kept set.
+FP2_DEVICE uint32_t pruned_word(const uint32_t* kmask, int base, int i) {
+  if (base >= i) return 0u;
+  const uint32_t kept = kmask[base >> 5];
+  const int nvalid = i - base;  // blocks base .. i-1 are candidates
+  const uint32_t lim = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
+  return ~kept & lim;
+}
+
+// Scaled logit (log2 domain) of one S element with the tile's mask applied.
+FP2_DEVICE float logit(uint32_t sbits, float scale_log2, bool virt, bool diag, uint32_t mword, int e, int col,
+                       int tl, float log2_blk) {
+  const float xv = __uint_as_float(sbits) * scale_log2;
+  if (virt) return ((mword >> e) & 1u) ? xv + log2_blk : -CUDART_INF_F;
+  if (diag && col > tl) return -CUDART_INF_F;
+  return xv;
+}
+
+// Bounded wait used only while draining in-flight copies at exit; ignores the abort flag.
+// Copies and MMAs complete within microseconds, so the limit is short.
+FP2_DEVICE void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) {
+      set_status(status, FP2_DEV_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int DT, int D, int BN>
+__global__ void __launch_bounds__(320, 1)
+    attention_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Fp2Plan P) {
+  using C = AttnCfg<DT, D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = kv_full + C::NSLOT;
+  uint64_t* s_full = kv_empty + C::NSLOT;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* mask_ready = o_done + 2;
+  uint64_t* mma_done = mask_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int r, i, sub;
+  if (!map_heavy_first(P, 1, a.Hkv * a.parts, blockIdx.x, r, i, sub)) return;
+  const int g = sub / a.parts, part = sub % a.parts;
+  const int L = P.len[r];
+  const int64_t row = static_cast<int64_t>(P.blk_off[r] + i) * a.Hkv + g;
+  const int rs = a.row_ptr[row], re = a.row_ptr[row + 1];
+  const int nkept = re - rs;
+  if (nkept <= 0 || nkept > i + 1) {
+    if (tid == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
+    return;
+  }
+  const int npruned = i + 1 - nkept;
+  const int n_virt = (a.mean_correction && npruned > 0) ? (i + BN - 1) / BN : 0;
+  const int n_tiles = n_virt + nkept;
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+      mbar_init(&o_done[s], 1);
+    }
+    for (int k = 0; k < C::NSLOT; ++k) {
+      mbar_init(&kv_full[k], 1);
+      mbar_init(&kv_empty[k], 1);
+    }
+    mbar_init(mask_ready, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    const int nw = (i + 32) / 32;
+    for (int w = lane; w < nw; w += 32) kmask[w] = 0u;
+    __syncwarp();
+    bool bad = false;
+    for (int e = lane; e < nkept; e += 32) {
+      const int j = a.col_idx[rs + e];
+      const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
+      if (j < 0 || j > i || j <= prev)
+        bad = true;
+      else
+        atomicOr(&kmask[j >> 5], 1u << (j & 31));
+    }
+    if (lane == 0 && a.col_idx[re - 1] != i) bad = true;
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(mask_ready);
+      tma_prefetch_desc(&a.tm_q);
+      tma_prefetch_desc(&a.tm_k);
+      tma_prefetch_desc(&a.tm_v);
+      tma_prefetch_desc(&a.tm_kb);
+      tma_prefetch_desc(&a.tm_vb);
+      constexpr int HS = 128 / BN;
+      const int tokq = P.tok_off[r] + i * BN;
+      for (int s = 0; s < a.NT; ++s) {
+        mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
+        for (int hs = 0; hs < HS; ++hs) {
+          const int hl = (part * a.NT + s) * HS + hs;
+          const int h = g * a.G + (hl % a.G);
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + c * (128 * 128) + hs * (BN * 128), &a.tm_q, &q_full[s],
+                        c * C::KCH, h, tokq);
+        }
+      }
+      int p = 0;
+      for (int jt = 0; jt < n_tiles && !*abort_flag; ++jt) {
+        int j = -1;
+        if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), i);
+        bool stop = false;
+        for (int kv = 0; kv < 2; ++kv) {
+          const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
+          if (wrap > 0 && !mbar_wait(&kv_empty[slot], (wrap - 1) & 1, abort_flag, a.status)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
+          uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
+          if (j < 0) {
+            const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
+            for (int c = 0; c < C::DCH; ++c)
+              tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.blk_off[r] + jt * BN);
+          } else if (a.page_table == nullptr) {
+            const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
+            for (int c = 0; c < C::DCH; ++c)
+              tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.tok_off[r] + j * BN);
+          } else {
+            const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
+            const int PR = min(BN, a.page_size);
+            for (int sb = 0; sb < BN / PR; ++sb) {
+              int t = j * BN + sb * PR;
+              if (t >= L) t = (L - 1) - ((L - 1) % PR);  // past the end: reload the last rows (masked)
+              int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + t / a.page_size];
+              if (page < 0 || page >= a.num_pages) {
+                set_status(a.status, FP2_DEV_PAGE_OOB);
+                page = 0;
+              }
+              const int flat = page * a.page_size + (t % a.page_size);
+              for (int c = 0; c < C::DCH; ++c)
+                tma_load_3d(dst + c * (BN * 128) + sb * (PR * 128), tm, &kv_full[slot], c * C::KCH, g, flat);
+            }
+          }
+          ++p;
+        }
+        if (stop) break;
+      }
+      // Never leave with copies in flight.
+      for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status);
+      for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status);
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int s = 0; s < a.NT && ok; ++s) ok = mbar_wait(&q_full[s], 0, abort_flag, a.status);
+      tc_fence_after();
+      int p = 0;
+      for (int jt = 0; jt < n_tiles && ok; ++jt) {
+        int slot = p % C::NSLOT;
+        if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t kaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
+        for (int s = 0; s < a.NT; ++s) {
+          if (jt > 0 && !mbar_wait(&o_done[s], (jt - 1) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qaddr = sbase + C::OFF_Q + s * C::Q_BYTES;
+          const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+#pragma unroll
+          for (int k = 0; k < D / C::UK; ++k) {
+            const int c = (k * C::UK) / C::KCH;
+            const int koff = ((k * C::UK) % C::KCH) * C::ELT;
+            const uint64_t ad = smem_desc_sw128(qaddr + c * (128 * 128) + koff, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(kaddr + c * (BN * 128) + koff, 16, 1024);
+            umma_ss<C::KIND>(dcol, ad, bd, C::IDESC_S, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[s]);
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[slot]);
+        ++p;
+        slot = p % C::NSLOT;
+        if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t vaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
+        for (int s = 0; s < a.NT; ++s) {
+          if (!mbar_wait(&p_full[s], jt & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+          const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
+#pragma unroll
+          for (int k = 0; k < BN / C::UK; ++k) {
+            const uint64_t bd = smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
+            umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&o_done[s]);
+        }
+        if (!ok) break;
+        umma_commit(&kv_empty[slot]);
+        ++p;
+      }
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0, a.status);
+    }
+  } else if (warp < 4 * a.NT) {
+    // ---------------------------------------------------------------- softmax / epilogue
+    const int s = warp >> 2, qd = warp & 3;
+    const int rt = qd * 32 + lane;
+    constexpr int HS = 128 / BN;
+    const int hs = rt / BN, tl = rt % BN;
+    const int hl = (part * a.NT + s) * HS + hs;
+    const bool row_ok = (hl < a.G) && (i * BN + tl < L);
+    const int h = g * a.G + min(hl, a.G - 1);
+    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + (s ? C::S_COL1 : C::S_COL0);
+    const uint32_t o_addr = tmem + lane_base + (s ? C::O_COL1 : C::O_COL0);
+    float m_run = -CUDART_INF_F, l_run = 0.f;
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status));
+    int done_tiles = 0;
+    for (int jt = 0; jt < n_tiles && ok; ++jt) {
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jt & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      // Kind of tile: virtual (pooled keys of blocks [jt*BN, jt*BN+BN)), diagonal, or full.
+      const bool virt = jt < n_virt;
+      const bool diag = !virt && jt == n_tiles - 1;
+      // Pass 1: masked row max of this tile, 32 columns at a time straight from TMEM.
+      float mt = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(s_addr + c * 32, v);
+        const uint32_t mword = virt ? pruned_word(kmask, jt * BN + c * 32, i) : 0u;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float xv = logit(v[e], a.sm_scale_log2, virt, diag, mword, e, c * 32 + e, tl, a.log2_blk);
+          mt = fmaxf(mt, xv);
+        }
+      }
+      const float m_new = fmaxf(m_run, mt);
+      const bool need = m_new > m_run + 8.0f;
+      if (jt > 0 && __any_sync(0xFFFFFFFFu, need)) {
+        const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32_sync(o_addr + c * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tmem_st32(o_addr + c * 32, v);
+        }
+        tmem_st_wait();
+      }
+      if (need) {
+        l_run = (m_run == -CUDART_INF_F) ? 0.f : l_run * fast_exp2(m_run - m_new);
+        m_run = m_new;
+      }
+      const float mu = (m_run == -CUDART_INF_F) ? 0.f : m_run;
+      // Pass 2: P = 2^(x - m), packed to the MMA type and written over the columns of S
+      // already consumed (chunk c of P lands at or before chunk c of S).
+      float rsum = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(s_addr + c * 32, v);
+        const uint32_t mword = virt ? pruned_word(kmask, jt * BN + c * 32, i) : 0u;
+        float pv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          pv[e] = fast_exp2(logit(v[e], a.sm_scale_log2, virt, diag, mword, e, c * 32 + e, tl, a.log2_blk) - mu);
+          rsum += pv[e];
+        }
+        if constexpr (DT == 1) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+          tmem_st16(s_addr + c * 16, pk);
+        } else if constexpr (DT == 2) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk[e] = pack_e4m3x4(pv[4 * e], pv[4 * e + 1], pv[4 * e + 2], pv[4 * e + 3]);
+          tmem_st8(s_addr + c * 8, pk);
+        } else {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(pv[e]);
+          tmem_st32(s_addr + c * 32, pk);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[s]);
+      l_run += rsum;
+      done_tiles = jt + 1;
+    }
+    if (ok && done_tiles == n_tiles)
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_tiles - 1) & 1, abort_flag, a.status));
+    tc_fence_after();
+    if (ok) {
+      const int tok = P.tok_off[r] + i * BN + tl;
+      const float inv = a.v_descale / l_run;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32_sync(o_addr + c * 32, v);
+        if (row_ok) {
+          if constexpr (DT == 0) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                                    (static_cast<int64_t>(tok) * a.Hq + h) * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                   __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                                  (static_cast<int64_t>(tok) * a.Hq + h) * D + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv, __uint_as_float(v[8 * e + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv);
+              dst[e] = w;
+            }
+          }
+        }
+      }
+      if (row_ok && a.lse != nullptr)
+        a.lse[static_cast<int64_t>(h) * a.total_tokens + tok] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+template <int DT, int D, int BN>
+static cudaError_t launch_one(const AttnArgs& a, const Fp2Plan& P, int64_t items, cudaStream_t stream) {
+  using C = AttnCfg<DT, D, BN>;
+  cudaError_t e = cudaFuncSetAttribute(attention_kernel<DT, D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  attention_kernel<DT, D, BN><<<static_cast<unsigned>(items), 320, C::SMEM_BYTES, stream>>>(a, P);
+  return cudaGetLastError();
+}
+
+size_t attention_smem_bytes(int dtype, int D, int B) {
+  if (dtype == FP2_F32 && D == 64 && B == 64) return AttnCfg<0, 64, 64>::SMEM_BYTES;
+  if (dtype == FP2_F32 && D == 64 && B == 128) return AttnCfg<0, 64, 128>::SMEM_BYTES;
+  if (dtype == FP2_BF16 && D == 64 && B == 64) return AttnCfg<1, 64, 64>::SMEM_BYTES;
+  if (dtype == FP2_BF16 && D == 64 && B == 128) return AttnCfg<1, 64, 128>::SMEM_BYTES;
+  if (dtype == FP2_BF16 && D == 128 && B == 64) return AttnCfg<1, 128, 64>::SMEM_BYTES;
+  if (dtype == FP2_BF16 && D == 128 && B == 128) return AttnCfg<1, 128, 128>::SMEM_BYTES;
+  if (dtype == FP2_E4M3 && D == 128 && B == 64) return AttnCfg<2, 128, 64>::SMEM_BYTES;
+  if (dtype == FP2_E4M3 && D == 128 && B == 128) return AttnCfg<2, 128, 128>::SMEM_BYTES;
+  return 0;
+}
+
+cudaError_t launch_attention(int dtype, int D, int B, const AttnArgs& a, const Fp2Plan& P, int64_t items,
+                             cudaStream_t stream) {
+  if (dtype == FP2_F32 && D == 64 && B == 64) return launch_one<0, 64, 64>(a, P, items, stream);
+  if (dtype == FP2_F32 && D == 64 && B == 128) return launch_one<0, 64, 128>(a, P, items, stream);
+  if (dtype == FP2_BF16 && D == 64 && B == 64) return launch_one<1, 64, 64>(a, P, items, stream);
+  if (dtype == FP2_BF16 && D == 64 && B == 128) return launch_one<1, 64, 128>(a, P, items, stream);
+  if (dtype == FP2_BF16 && D == 128 && B == 64) return launch_one<1, 128, 64>(a, P, items, stream);
+  if (dtype == FP2_BF16 && D == 128 && B == 128) return launch_one<1, 128, 128>(a, P, items, stream);
+  if (dtype == FP2_E4M3 && D == 128 && B == 64) return launch_one<2, 128, 64>(a, P, items, stream);
+  if (dtype == FP2_E4M3 && D == 128 && B == 128) return launch_one<2, 128, 128>(a, P, items, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fp2

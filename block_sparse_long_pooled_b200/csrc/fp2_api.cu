@@ -1,0 +1,440 @@
+// Host side of the C ABI declared in include/fp2.h: argument validation, the launch plan,
+// workspace sizing, TMA descriptor encoding and kernel launches.  Allocates nothing and
+// never synchronises the caller's stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/fp2.h"
+#include "fp2_kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fp2_status fail(fp2_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+fp2_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FP2_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : (t == FP2_BF16 ? 2 : 1); }
+
+// Everything derived from (problem, params) on the host.
+struct Ctx {
+  Fp2Plan plan;
+  int elt = 0, G = 0, W = 0;
+  int64_t T = 0, total_blocks = 0, rows = 0, cap = 0;
+  float scale = 0.f;
+  fp2_workspace ws{};
+  size_t off_bitmask = 0, off_counts = 0;  // inside scratch
+  // fp2_prefill carve-outs (offsets after scratch_bytes)
+  size_t off_qbar = 0, off_kbar = 0, off_vbar = 0, off_kbm = 0, off_vbm = 0, off_rowptr = 0, off_colidx = 0;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
+  if (p == nullptr || s == nullptr) return fail(FP2_ERR_INVALID_ARG, "problem and params must not be NULL");
+  if (p->num_seqs < 1 || p->num_seqs > FP2_MAX_SEQS)
+    return fail(FP2_ERR_UNSUPPORTED, "num_seqs must be in [1, FP2_MAX_SEQS]");
+  if (p->cu_seqlens_q_host == nullptr) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens_q_host is NULL");
+  if (p->dtype != FP2_F32 && p->dtype != FP2_BF16 && p->dtype != FP2_E4M3)
+    return fail(FP2_ERR_INVALID_ARG, "unknown dtype");
+  if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_q_heads % p->num_kv_heads != 0)
+    return fail(FP2_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
+  c.G = p->num_q_heads / p->num_kv_heads;
+  if (c.G > 32) return fail(FP2_ERR_UNSUPPORTED, "GQA group size above 32");
+  if (p->head_dim != 64 && p->head_dim != 128) return fail(FP2_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (p->dtype == FP2_F32 && p->head_dim != 64) return fail(FP2_ERR_UNSUPPORTED, "F32 inputs need head_dim 64");
+  if (p->dtype == FP2_E4M3 && p->head_dim != 128) return fail(FP2_ERR_UNSUPPORTED, "E4M3 inputs need head_dim 128");
+  if (s->block_size != 64 && s->block_size != 128) return fail(FP2_ERR_UNSUPPORTED, "block_size must be 64 or 128");
+  if (!(s->alpha >= 0.f && s->alpha <= 1.f)) return fail(FP2_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (s->sink_blocks < 0 || s->window_blocks < 0 || s->last_n_blocks < 0 || s->min_sparse_len < 0)
+    return fail(FP2_ERR_INVALID_ARG, "sink/window/last_n/min_sparse_len must be >= 0");
+  if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale))
+    return fail(FP2_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  for (float d : {p->q_descale, p->k_descale, p->v_descale})
+    if (!(d > 0.f) || !std::isfinite(d)) return fail(FP2_ERR_INVALID_ARG, "descale factors must be finite and > 0");
+  c.elt = elt_bytes(p->dtype);
+  const int B = s->block_size, D = p->head_dim, Hq = p->num_q_heads, Hkv = p->num_kv_heads;
+
+  const int32_t* cq = p->cu_seqlens_q_host;
+  const int32_t* ck = p->cu_seqlens_k_host ? p->cu_seqlens_k_host : cq;
+  if (cq[0] != 0 || ck[0] != 0) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens must start at 0");
+  Fp2Plan& P = c.plan;
+  std::memset(&P, 0, sizeof(P));
+  P.num_seqs = p->num_seqs;
+  int64_t T = 0, blocks = 0, cap = 0;
+  int max_nblk = 0;
+  for (int r = 0; r < p->num_seqs; ++r) {
+    const int64_t Lq = static_cast<int64_t>(cq[r + 1]) - cq[r];
+    const int64_t Lk = static_cast<int64_t>(ck[r + 1]) - ck[r];
+    if (Lq < 0 || Lk < 0) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing");
+    if (Lq != Lk || cq[r] != ck[r])
+      return fail(FP2_ERR_UNSUPPORTED, "q_len != kv_len (chunked prefill) is not supported");
+    const int64_t N = (Lq + B - 1) / B;
+    if (N > FP2_MAX_BLOCKS) return fail(FP2_ERR_UNSUPPORTED, "a sequence has more than FP2_MAX_BLOCKS blocks");
+    P.tok_off[r] = cq[r];
+    P.len[r] = static_cast<int32_t>(Lq);
+    P.blk_off[r] = static_cast<int32_t>(blocks);
+    P.nblk[r] = static_cast<int32_t>(N);
+    T += Lq;
+    blocks += N;
+    cap += static_cast<int64_t>(Hkv) * N * (N + 1) / 2;
+    max_nblk = std::max<int>(max_nblk, static_cast<int>(N));
+  }
+  if (T != cq[p->num_seqs]) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens inconsistent");
+  if (T >= (int64_t(1) << 31) || cap >= (int64_t(1) << 31) || blocks * Hkv >= (int64_t(1) << 31))
+    return fail(FP2_ERR_UNSUPPORTED, "problem too large for 32-bit token / index offsets");
+  P.total_tokens = static_cast<int32_t>(T);
+  P.total_blocks = static_cast<int32_t>(blocks);
+  P.max_nblk = max_nblk;
+  for (int r = 0; r < p->num_seqs; ++r) P.sorted[r] = static_cast<int16_t>(r);
+  std::stable_sort(P.sorted, P.sorted + p->num_seqs, [&](int16_t x, int16_t y) { return P.nblk[x] > P.nblk[y]; });
+  c.T = T;
+  c.total_blocks = blocks;
+  c.rows = blocks * Hkv;
+  c.cap = cap;
+  c.W = std::max(1, (max_nblk + 31) / 32);
+  c.scale = p->softmax_scale > 0.f ? p->softmax_scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+
+  // Tensors (only checked when there is data to read).
+  if (T > 0) {
+    if (p->q == nullptr || p->k == nullptr || p->v == nullptr) return fail(FP2_ERR_INVALID_ARG, "q/k/v must not be NULL");
+    if (!aligned16(p->q) || !aligned16(p->k) || !aligned16(p->v))
+      return fail(FP2_ERR_INVALID_ARG, "q/k/v must be 16-byte aligned");
+    if (p->q_stride_tok < static_cast<int64_t>(Hq) * D || p->kv_stride_tok < static_cast<int64_t>(Hkv) * D)
+      return fail(FP2_ERR_INVALID_ARG, "token strides must be >= heads * head_dim");
+    if ((p->q_stride_tok * c.elt) % 16 != 0 || (p->kv_stride_tok * c.elt) % 16 != 0)
+      return fail(FP2_ERR_INVALID_ARG, "token strides must be multiples of 16 bytes");
+    if (p->page_table != nullptr) {
+      const int ps = p->page_size;
+      if (ps < 16 || (ps & (ps - 1)) != 0) return fail(FP2_ERR_UNSUPPORTED, "page_size must be a power of two >= 16");
+      if (p->num_pages <= 0 || static_cast<int64_t>(p->num_pages) * ps >= (int64_t(1) << 31))
+        return fail(FP2_ERR_INVALID_ARG, "num_pages out of range");
+      for (int r = 0; r < p->num_seqs; ++r)
+        if ((P.len[r] + ps - 1) / ps > p->max_pages_per_seq)
+          return fail(FP2_ERR_INVALID_ARG, "max_pages_per_seq too small for a sequence");
+    }
+  }
+
+  fp2_workspace& w = c.ws;
+  w.total_tokens = T;
+  w.total_blocks = blocks;
+  w.index_rows = c.rows;
+  w.col_capacity = cap;
+  w.qbar_bytes = static_cast<size_t>(blocks) * Hq * D * 4;
+  w.kbar_bytes = static_cast<size_t>(blocks) * Hkv * D * 4;
+  w.vbar_bytes = w.kbar_bytes;
+  w.kbar_mma_bytes = static_cast<size_t>(blocks) * Hkv * D * c.elt;
+  w.vbar_mma_bytes = w.kbar_mma_bytes;
+  w.row_ptr_bytes = static_cast<size_t>(c.rows + 1) * 4;
+  w.col_idx_bytes = static_cast<size_t>(std::max<int64_t>(cap, 1)) * 4;
+  c.off_bitmask = FP2_SCRATCH_STATUS_BYTES;
+  c.off_counts = c.off_bitmask + align_up(static_cast<size_t>(c.rows) * c.W * 4);
+  w.scratch_bytes = c.off_counts + align_up(static_cast<size_t>(c.rows) * 4);
+  size_t o = w.scratch_bytes;
+  c.off_qbar = o;   o += align_up(w.qbar_bytes);
+  c.off_kbar = o;   o += align_up(w.kbar_bytes);
+  c.off_vbar = o;   o += align_up(w.vbar_bytes);
+  c.off_kbm = o;    o += align_up(w.kbar_mma_bytes);
+  c.off_vbm = o;    o += align_up(w.vbar_mma_bytes);
+  c.off_rowptr = o; o += align_up(w.row_ptr_bytes);
+  c.off_colidx = o; o += align_up(w.col_idx_bytes);
+  w.prefill_scratch_bytes = o;
+  return FP2_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D map over a token-major tensor: dims {d, heads, rows}, box {128B/elt, 1, box_rows}, 128B swizzle.
+fp2_status encode_3d(CUtensorMap* m, fp2_dtype dt, const void* base, int D, int heads, int64_t rows,
+                     int64_t row_stride_elems, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (fn == nullptr) return fail(FP2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const int elt = elt_bytes(dt);
+  const CUtensorMapDataType t = dt == FP2_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dt == FP2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(std::max<int64_t>(rows, 1))};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elt, static_cast<cuuint64_t>(row_stride_elems) * elt};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elt), 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(m, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FP2_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
+  return FP2_OK;
+}
+
+uint32_t* status_ptr(void* scratch) { return static_cast<uint32_t*>(scratch); }
+
+fp2_status check_scratch(const void* scratch, size_t have, size_t need) {
+  if (scratch == nullptr) return fail(FP2_ERR_INVALID_ARG, "scratch is NULL");
+  if ((reinterpret_cast<uintptr_t>(scratch) & (kAlign - 1)) != 0)
+    return fail(FP2_ERR_INVALID_ARG, "scratch must be 256-byte aligned");
+  if (have < need)
+    return fail(FP2_ERR_WORKSPACE_TOO_SMALL,
+                "scratch_bytes " + std::to_string(have) + " < required " + std::to_string(need));
+  return FP2_OK;
+}
+
+fp2_status check_pooled(const fp2_pooled* pl, bool need_q) {
+  if (pl == nullptr) return fail(FP2_ERR_INVALID_ARG, "pooled is NULL");
+  if ((need_q && pl->qbar == nullptr) || pl->kbar == nullptr || pl->vbar == nullptr || pl->kbar_mma == nullptr ||
+      pl->vbar_mma == nullptr)
+    return fail(FP2_ERR_INVALID_ARG, "pooled buffers must not be NULL");
+  const void* bufs[5] = {pl->qbar, pl->kbar, pl->vbar, pl->kbar_mma, pl->vbar_mma};
+  for (const void* q : bufs)
+    if (q != nullptr && !aligned16(q)) return fail(FP2_ERR_INVALID_ARG, "pooled buffers must be 16-byte aligned");
+  return FP2_OK;
+}
+
+fp2_status check_index(const fp2_index* ix, const Ctx& c) {
+  if (ix == nullptr || ix->row_ptr == nullptr || ix->col_idx == nullptr)
+    return fail(FP2_ERR_INVALID_ARG, "index buffers must not be NULL");
+  if (ix->col_capacity < 0) return fail(FP2_ERR_INVALID_ARG, "col_capacity must be >= 0");
+  (void)c;
+  return FP2_OK;
+}
+
+fp2_status run_pool(const fp2_problem* p, const fp2_sparse_params* s, const Ctx& c, const fp2_pooled* pl,
+                    void* scratch, cudaStream_t st) {
+  fp2::PoolArgs a{};
+  a.q = p->q;
+  a.k = p->k;
+  a.v = p->v;
+  a.q_stride = p->q_stride_tok;
+  a.kv_stride = p->kv_stride_tok;
+  a.page_table = p->page_table;
+  a.page_size = p->page_size;
+  a.max_pages = p->max_pages_per_seq;
+  a.num_pages = p->num_pages;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.D = p->head_dim;
+  a.B = s->block_size;
+  a.q_descale = p->q_descale;
+  a.k_descale = p->k_descale;
+  a.v_descale = p->v_descale;
+  a.qbar = pl->qbar;
+  a.kbar = pl->kbar;
+  a.vbar = pl->vbar;
+  a.kbar_mma = pl->kbar_mma;
+  a.vbar_mma = pl->vbar_mma;
+  a.status = status_ptr(scratch);
+  const cudaError_t e = fp2::launch_pool(p->dtype, a, c.plan, st);
+  return e == cudaSuccess ? FP2_OK : cuda_fail(e, "pool kernel launch");
+}
+
+fp2_status run_discover(const fp2_problem* p, const fp2_sparse_params* s, const Ctx& c, const fp2_pooled* pl,
+                        const fp2_index* ix, void* scratch, cudaStream_t st) {
+  fp2::DiscArgs a{};
+  a.qbar = pl->qbar;
+  a.kbar = pl->kbar;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = c.G;
+  a.D = p->head_dim;
+  a.scale = c.scale;
+  a.dense_all = s->alpha <= 0.f ? 1 : 0;
+  a.ln_alpha = s->alpha > 0.f ? static_cast<float>(std::log(static_cast<double>(s->alpha))) : 0.f;
+  a.sink = s->sink_blocks;
+  a.window = s->window_blocks;
+  a.last_n = s->last_n_blocks;
+  a.min_sparse_len = s->min_sparse_len;
+  a.SP = std::max(32, (c.plan.max_nblk + 31) / 32 * 32);
+  // Largest tile of query blocks whose scores fit in shared memory (TI * G <= 32 rows).
+  int TI = std::max(1, 32 / c.G);
+  while (TI > 1 && fp2::discover_smem_bytes(a.D, c.G, TI, a.SP) > 200 * 1024) --TI;
+  if (fp2::discover_smem_bytes(a.D, c.G, TI, a.SP) > 220 * 1024)
+    return fail(FP2_ERR_UNSUPPORTED, "group size x blocks per sequence too large for discovery");
+  a.TI = TI;
+  a.W = c.W;
+  a.bitmask = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + c.off_bitmask);
+  a.counts = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + c.off_counts);
+  a.status = status_ptr(scratch);
+  int64_t items = 0;
+  for (int r = 0; r < c.plan.num_seqs; ++r) items += static_cast<int64_t>((c.plan.nblk[r] + TI - 1) / TI) * a.Hkv;
+  if (items == 0) return FP2_OK;
+  const cudaError_t e = fp2::launch_discover(a, c.plan, items, c.rows, ix->row_ptr, ix->col_idx, ix->col_capacity, st);
+  return e == cudaSuccess ? FP2_OK : cuda_fail(e, "discover kernels launch");
+}
+
+fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ctx& c, const fp2_pooled* pl,
+                      const fp2_index* ix, void* out, float* lse, void* scratch, cudaStream_t st) {
+  const int B = s->block_size, D = p->head_dim;
+  if (fp2::attention_smem_bytes(p->dtype, D, B) == 0)
+    return fail(FP2_ERR_UNSUPPORTED, "no attention kernel for this (dtype, head_dim, block_size)");
+  fp2::AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
+  fp2_status st2;
+  const bool paged = p->page_table != nullptr;
+  if ((st2 = encode_3d(&a.tm_q, p->dtype, p->q, D, p->num_q_heads, c.T, p->q_stride_tok, B)) != FP2_OK) return st2;
+  const int64_t kv_rows = paged ? static_cast<int64_t>(p->num_pages) * p->page_size : c.T;
+  const int kv_box = paged ? std::min(B, p->page_size) : B;
+  if ((st2 = encode_3d(&a.tm_k, p->dtype, p->k, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box)) != FP2_OK)
+    return st2;
+  if ((st2 = encode_3d(&a.tm_v, p->dtype, p->v, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box)) != FP2_OK)
+    return st2;
+  const int64_t hd = static_cast<int64_t>(p->num_kv_heads) * D;
+  if ((st2 = encode_3d(&a.tm_kb, p->dtype, pl->kbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B)) != FP2_OK)
+    return st2;
+  if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B)) != FP2_OK)
+    return st2;
+  a.row_ptr = ix->row_ptr;
+  a.col_idx = ix->col_idx;
+  a.page_table = p->page_table;
+  a.page_size = p->page_size;
+  a.max_pages = p->max_pages_per_seq;
+  a.num_pages = p->num_pages;
+  a.out = out;
+  a.lse = lse;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.G = c.G;
+  const int mtiles = (c.G * B + 127) / 128;
+  a.NT = mtiles >= 2 ? 2 : 1;
+  a.parts = (mtiles + a.NT - 1) / a.NT;
+  a.sm_scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634 *
+                                       static_cast<double>(p->q_descale) * static_cast<double>(p->k_descale));
+  a.v_descale = p->v_descale;
+  a.log2_blk = static_cast<float>(std::log2(static_cast<double>(B)));
+  a.mean_correction = s->mean_correction ? 1 : 0;
+  a.total_tokens = static_cast<int>(c.T);
+  a.status = status_ptr(scratch);
+  const int64_t items = c.total_blocks * p->num_kv_heads * a.parts;
+  if (items == 0) return FP2_OK;
+  const cudaError_t e = fp2::launch_attention(p->dtype, D, B, a, c.plan, items, st);
+  return e == cudaSuccess ? FP2_OK : cuda_fail(e, "attention kernel launch");
+}
+
+fp2_status clear_status(void* scratch, cudaStream_t st) {
+  const cudaError_t e = cudaMemsetAsync(scratch, 0, FP2_SCRATCH_STATUS_BYTES, st);
+  return e == cudaSuccess ? FP2_OK : cuda_fail(e, "status reset");
+}
+
+}  // namespace
+
+extern "C" {
+
+fp2_status fp2_workspace_query(const fp2_problem* problem, const fp2_sparse_params* params, fp2_workspace* out) {
+  if (out == nullptr) return fail(FP2_ERR_INVALID_ARG, "out is NULL");
+  Ctx c;
+  const fp2_status s = validate(problem, params, c);
+  if (s != FP2_OK) return s;
+  *out = c.ws;
+  g_last_error.clear();
+  return FP2_OK;
+}
+
+fp2_status fp2_pool(const fp2_problem* problem, const fp2_sparse_params* params, const fp2_pooled* pooled,
+                    void* scratch, size_t scratch_bytes, fp2_stream_t stream) {
+  Ctx c;
+  fp2_status s;
+  if ((s = validate(problem, params, c)) != FP2_OK) return s;
+  if ((s = check_scratch(scratch, scratch_bytes, c.ws.scratch_bytes)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, true)) != FP2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_status(scratch, st)) != FP2_OK) return s;
+  if (c.T == 0) return FP2_OK;
+  return run_pool(problem, params, c, pooled, scratch, st);
+}
+
+fp2_status fp2_discover(const fp2_problem* problem, const fp2_sparse_params* params, const fp2_pooled* pooled,
+                        const fp2_index* index, void* scratch, size_t scratch_bytes, fp2_stream_t stream) {
+  Ctx c;
+  fp2_status s;
+  if ((s = validate(problem, params, c)) != FP2_OK) return s;
+  if ((s = check_scratch(scratch, scratch_bytes, c.ws.scratch_bytes)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, true)) != FP2_OK) return s;
+  if ((s = check_index(index, c)) != FP2_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_status(scratch, st)) != FP2_OK) return s;
+  if (c.T == 0) return FP2_OK;
+  return run_discover(problem, params, c, pooled, index, scratch, st);
+}
+
+fp2_status fp2_attend(const fp2_problem* problem, const fp2_sparse_params* params, const fp2_pooled* pooled,
+                      const fp2_index* index, void* out, float* lse, void* scratch, size_t scratch_bytes,
+                      fp2_stream_t stream) {
+  Ctx c;
+  fp2_status s;
+  if ((s = validate(problem, params, c)) != FP2_OK) return s;
+  if ((s = check_scratch(scratch, scratch_bytes, c.ws.scratch_bytes)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, false)) != FP2_OK) return s;
+  if ((s = check_index(index, c)) != FP2_OK) return s;
+  if (out == nullptr || !aligned16(out)) return fail(FP2_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_status(scratch, st)) != FP2_OK) return s;
+  if (c.T == 0) return FP2_OK;
+  return run_attend(problem, params, c, pooled, index, out, lse, scratch, st);
+}
+
+fp2_status fp2_prefill(const fp2_problem* problem, const fp2_sparse_params* params, void* out, float* lse,
+                       void* scratch, size_t scratch_bytes, fp2_stream_t stream) {
+  Ctx c;
+  fp2_status s;
+  if ((s = validate(problem, params, c)) != FP2_OK) return s;
+  if ((s = check_scratch(scratch, scratch_bytes, c.ws.prefill_scratch_bytes)) != FP2_OK) return s;
+  if (out == nullptr || !aligned16(out)) return fail(FP2_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
+  char* base = static_cast<char*>(scratch);
+  fp2_pooled pl{reinterpret_cast<float*>(base + c.off_qbar), reinterpret_cast<float*>(base + c.off_kbar),
+                reinterpret_cast<float*>(base + c.off_vbar), base + c.off_kbm, base + c.off_vbm};
+  fp2_index ix{reinterpret_cast<int32_t*>(base + c.off_rowptr), reinterpret_cast<int32_t*>(base + c.off_colidx),
+               std::max<int64_t>(c.cap, 1)};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = clear_status(scratch, st)) != FP2_OK) return s;
+  if (c.T == 0) return FP2_OK;
+  if ((s = run_pool(problem, params, c, &pl, scratch, st)) != FP2_OK) return s;
+  if ((s = run_discover(problem, params, c, &pl, &ix, scratch, st)) != FP2_OK) return s;
+  return run_attend(problem, params, c, &pl, &ix, out, lse, scratch, st);
+}
+
+fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_out) {
+  if (scratch == nullptr || status_out == nullptr) return fail(FP2_ERR_INVALID_ARG, "NULL argument");
+  uint32_t w = 0;
+  const cudaError_t e = cudaMemcpy(&w, scratch, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  *status_out = w;
+  if (w & FP2_DEV_TIMEOUT) return fail(FP2_ERR_TIMEOUT, "a device-side wait timed out");
+  if (w & (FP2_DEV_PAGE_OOB | FP2_DEV_INDEX_OOB | FP2_DEV_CAPACITY))
+    return fail(FP2_ERR_DEVICE_BOUNDS, "device reported an out-of-range page id, index entry or capacity overflow");
+  return FP2_OK;
+}
+
+const char* fp2_last_error(void) { return g_last_error.c_str(); }
+
+int32_t fp2_version(void) { return 10000; }
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// Kernel argument blocks and launchers (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fp2_plan.h"
+
+namespace fp2 {
+
+struct PoolArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t q_stride, kv_stride;  // elements between tokens
+  const int32_t* page_table;    // NULL -> contiguous K/V
+  int page_size, max_pages, num_pages;
+  int Hq, Hkv, D, B;
+  float q_descale, k_descale, v_descale;
+  float* qbar;
+  float* kbar;
+  float* vbar;
+  void* kbar_mma;
+  void* vbar_mma;
+  uint32_t* status;
+};
+
+struct DiscArgs {
+  const float* qbar;
+  const float* kbar;
+  int Hq, Hkv, G, D;
+  float scale;      // softmax scale used for the block scores
+  float ln_alpha;   // natural log of alpha (alpha > 0)
+  int dense_all;    // alpha <= 0: keep everything
+  int sink, window, last_n, min_sparse_len;
+  int TI;           // query blocks per CTA (TI * G <= 32)
+  int SP;           // padded score row length (>= max N, multiple of 32)
+  int W;            // bitmask words per row
+  uint32_t* bitmask;
+  int32_t* counts;
+  uint32_t* status;
+};
+
+struct AttnArgs {
+  CUtensorMap tm_q;   // Q  [T, Hq, d]       box {128B / elt, 1, B}
+  CUtensorMap tm_k;   // K  tokens (flat)    box {128B / elt, 1, B or page rows}
+  CUtensorMap tm_v;
+  CUtensorMap tm_kb;  // kbar_mma [blocks, Hkv, d] box {128B / elt, 1, B}
+  CUtensorMap tm_vb;
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const int32_t* page_table;  // NULL -> contiguous
+  int page_size, max_pages, num_pages;
+  void* out;                  // [T, Hq, d] bf16 (f32 for f32 inputs)
+  float* lse;                 // [Hq, T] or NULL
+  int Hq, Hkv, G;
+  int NT;                     // M tiles (128 packed rows each) per CTA: 1 or 2
+  int parts;                  // CTAs per (sequence, query block, KV head)
+  float sm_scale_log2;        // softmax scale * log2(e) * q_descale * k_descale
+  float v_descale;
+  float log2_blk;             // log2 of a pruned block's token count
+  int mean_correction;
+  int total_tokens;
+  uint32_t* status;
+};
+
+cudaError_t launch_pool(int dtype, const PoolArgs& a, const Fp2Plan& P, cudaStream_t stream);
+size_t discover_smem_bytes(int D, int G, int TI, int SP);
+cudaError_t launch_discover(const DiscArgs& a, const Fp2Plan& P, int64_t items, int64_t rows, int32_t* row_ptr,
+                            int32_t* col_idx, int64_t capacity, cudaStream_t stream);
+// Returns cudaErrorInvalidValue when no kernel exists for (dtype, d, B).
+cudaError_t launch_attention(int dtype, int D, int B, const AttnArgs& a, const Fp2Plan& P, int64_t items,
+                             cudaStream_t stream);
+size_t attention_smem_bytes(int dtype, int D, int B);
+
+}  // namespace fp2

@@ -1,0 +1,173 @@
+// Stage 1a: block-mean pooling of Q, K and V (FlashPrefill V2 paper page, Figure 3:
+// Stage 1 "pools block-mean statistics"; ResearchPod episode: a block is scored from a
+// simple average of its tokens).
+//
+// One pass over Q, K and V.  A CTA owns one pooled block b (B consecutive tokens of one
+// sequence) and a 256-vector slice of the concatenated token row [Q row | K row | V row];
+// each thread owns one 16-byte column vector of that row and walks the block's tokens
+// with eight independent 16-byte streaming loads in flight, accumulating in fp32.  Paged
+// K/V rows are gathered through the page table.  HBM-bound: the only traffic is one read
+// of Q, K, V and a (1/B)-sized write of the means.
+#include "fp2_device.cuh"
+#include "fp2_kernels.h"
+
+namespace fp2 {
+
+template <int DT>
+struct Elt;
+template <>
+struct Elt<0> {  // f32
+  static constexpr int kBytes = 4;
+};
+template <>
+struct Elt<1> {  // bf16
+  static constexpr int kBytes = 2;
+};
+template <>
+struct Elt<2> {  // e4m3
+  static constexpr int kBytes = 1;
+};
+
+FP2_DEVICE uint4 ld_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+template <int DT>
+FP2_DEVICE void accumulate(const uint4& v, float* acc) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if constexpr (DT == 0) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += __uint_as_float(w[e]);
+  } else if constexpr (DT == 1) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __uint_as_float(w[e] << 16);
+      acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((w[e] >> (16 * hlf)) & 0xFFFFu);
+        const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+        acc[4 * e + 2 * hlf] += f.x;
+        acc[4 * e + 2 * hlf + 1] += f.y;
+      }
+    }
+  }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Plan P) {
+  constexpr int VEC = 16 / Elt<DT>::kBytes;  // elements per 16-byte vector
+  const int b = blockIdx.x;
+  const int r = seq_of_block(P, b);
+  const int i = b - P.blk_off[r];
+  const int L = P.len[r];
+  const int t0 = i * a.B;
+  const int n = min(a.B, L - t0);
+  const int VQ = a.Hq * a.D / VEC, VK = a.Hkv * a.D / VEC;
+  const int vid = blockIdx.y * blockDim.x + threadIdx.x;
+  if (vid >= VQ + 2 * VK || n <= 0) return;
+
+  int which, col;
+  if (vid < VQ) {
+    which = 0;
+    col = vid * VEC;
+  } else if (vid < VQ + VK) {
+    which = 1;
+    col = (vid - VQ) * VEC;
+  } else {
+    which = 2;
+    col = (vid - VQ - VK) * VEC;
+  }
+  const char* base = static_cast<const char*>(which == 0 ? a.q : (which == 1 ? a.k : a.v));
+  const int64_t stride = which == 0 ? a.q_stride : a.kv_stride;
+  const bool paged = (which != 0) && (a.page_table != nullptr);
+  const int64_t tok_base = P.tok_off[r] + t0;
+
+  float acc[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+
+  for (int t = 0; t < n; t += 8) {
+    uint4 buf[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int tt = t + u;
+      if (tt < n) {
+        int64_t rowidx;
+        if (paged) {
+          const int tl = t0 + tt;
+          int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + tl / a.page_size];
+          if (page < 0 || page >= a.num_pages) {
+            set_status(a.status, FP2_DEV_PAGE_OOB);
+            page = 0;
+          }
+          rowidx = static_cast<int64_t>(page) * a.page_size + (tl % a.page_size);
+        } else {
+          rowidx = tok_base + tt;
+        }
+        buf[u] = ld_stream_v4(base + (rowidx * stride + col) * Elt<DT>::kBytes);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (t + u < n) accumulate<DT>(buf[u], acc);
+  }
+
+  const float descale = which == 0 ? a.q_descale : (which == 1 ? a.k_descale : a.v_descale);
+  const float fn = static_cast<float>(n);
+  float mean_raw[VEC];
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) mean_raw[e] = acc[e] / fn;
+
+  const int H = which == 0 ? a.Hq : a.Hkv;
+  float* dst = which == 0 ? a.qbar : (which == 1 ? a.kbar : a.vbar);
+  float4* d4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(b) * H * a.D + col);
+#pragma unroll
+  for (int e = 0; e < VEC / 4; ++e)
+    d4[e] = make_float4(mean_raw[4 * e] * descale, mean_raw[4 * e + 1] * descale, mean_raw[4 * e + 2] * descale,
+                        mean_raw[4 * e + 3] * descale);
+
+  if (which != 0) {
+    // Narrow copy in the MMA operand type (E4M3 stays in the stored, un-descaled domain).
+    char* nb = static_cast<char*>(which == 1 ? a.kbar_mma : a.vbar_mma);
+    uint4 out;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&out);
+    if constexpr (DT == 0) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ow[e] = __float_as_uint(mean_raw[e]);
+    } else if constexpr (DT == 1) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ow[e] = pack_bf16x2(mean_raw[2 * e], mean_raw[2 * e + 1]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        ow[e] = pack_e4m3x4(mean_raw[4 * e], mean_raw[4 * e + 1], mean_raw[4 * e + 2], mean_raw[4 * e + 3]);
+    }
+    *reinterpret_cast<uint4*>(nb + (static_cast<int64_t>(b) * H * a.D + col) * Elt<DT>::kBytes) = out;
+  }
+}
+
+cudaError_t launch_pool(int dtype, const PoolArgs& a, const Fp2Plan& P, cudaStream_t stream) {
+  const int elt = dtype == FP2_F32 ? 4 : (dtype == FP2_BF16 ? 2 : 1);
+  const int vec = 16 / elt;
+  const int nvec = (a.Hq + 2 * a.Hkv) * a.D / vec;
+  dim3 grid(P.total_blocks, (nvec + 255) / 256);
+  if (dtype == FP2_F32)
+    pool_kernel<0><<<grid, 256, 0, stream>>>(a, P);
+  else if (dtype == FP2_BF16)
+    pool_kernel<1><<<grid, 256, 0, stream>>>(a, P);
+  else
+    pool_kernel<2><<<grid, 256, 0, stream>>>(a, P);
+  return cudaGetLastError();
+}
+
+}  // namespace fp2

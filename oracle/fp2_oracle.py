@@ -209,7 +209,8 @@ def kept_from_csr(row_ptr, col_idx, seqlens, B, Hkv):
 
 
 def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correction: bool,
-           rows: Optional[np.ndarray] = None):
+           rows: Optional[np.ndarray] = None, head_ids: Optional[Sequence[int]] = None,
+           group: Optional[int] = None):
     """Exact attention over kept blocks plus mean correction for pruned ones, one sequence.
 
     Figure 4 caption: selected blocks are computed exactly; each pruned block J
@@ -225,11 +226,14 @@ def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correct
     q: [L, Hq, d]; k, v: [L, Hkv, d]; kbar, vbar: [N, Hkv, d]; counts: [N];
     kept: [Hkv, N, N].  rows: optional int array [n, 2] of (t, h) pairs; when
     given only those outputs are computed and O is [n, d], LSE [n].
-    Otherwise O is [L, Hq, d] and LSE [Hq, L].
+    Otherwise O is [L, Hq, d] and LSE [Hq, L].  head_ids / group: when q holds
+    only some query heads, head_ids[x] is the global head of q[:, x] and group
+    is G; rows then index q's own head axis.
     """
     L, Hq, d = q.shape
     Hkv = k.shape[1]
-    G = Hq // Hkv
+    G = group if group is not None else Hq // Hkv
+    gid = (lambda x: int(head_ids[x]) // G) if head_ids is not None else (lambda x: x // G)
     N = num_blocks(L, B)
     logn = np.log(counts.astype(np.float64))
     if rows is None:
@@ -248,7 +252,7 @@ def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correct
                 sel = sel_h[blocks == i]
                 work.append((int(h), int(i), rows[sel, 0], sel))
     for h, i, toks, dest in work:
-        g = h // G
+        g = gid(h)
         if not kept[g, i, i]:
             raise ValueError("the diagonal block must be kept (it is only partly visible)")
         kj = np.nonzero(kept[g, i, : i + 1])[0]

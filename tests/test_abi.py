@@ -1,0 +1,120 @@
+"""The C ABI library without a GPU: it loads, exports what include/fp2.h declares, and its
+host-side validation and workspace sizing behave (no CUDA call is made by these paths)."""
+
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_pooled_b200 import build as B
+from block_sparse_long_pooled_b200 import fp2
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    B.build()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "fp2.h")).read()
+    return sorted(set(re.findall(r"FP2_API\s+[\w\s\*]+?\b(fp2_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    decl = declared_functions()
+    assert decl == sorted(fp2.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB], capture_output=True, text=True, check=True).stdout
+    exported = sorted(l.split()[-1] for l in out.splitlines() if " T " in l)
+    assert exported == decl
+    lib = fp2.load_library()
+    for name in decl:
+        assert hasattr(lib, name)
+    assert fp2.fp2_version() == 10000
+
+
+def _problem(seqlens=(1000, 333), Hq=8, Hkv=2, d=128, dtype=torch.bfloat16, paged=False, page_size=64):
+    T = sum(seqlens)
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
+    q = torch.empty((T, Hq, d), dtype=dtype)
+    if paged:
+        npages = sum(-(-L // page_size) for L in seqlens)
+        k = torch.empty((npages, page_size, Hkv, d), dtype=dtype)
+        v = torch.empty_like(k)
+        pt = torch.zeros((len(seqlens), max(-(-L // page_size) for L in seqlens)), dtype=torch.int32)
+        return fp2.make_problem(q, k, v, cu, Hkv, page_table=pt)
+    k = torch.empty((T, Hkv, d), dtype=dtype)
+    v = torch.empty_like(k)
+    return fp2.make_problem(q, k, v, cu, Hkv)
+
+
+def test_workspace_sizes():
+    prob = _problem()
+    ws = fp2.fp2_workspace_query(prob, fp2.make_params(128))
+    N = [8, 3]
+    assert ws.total_tokens == 1333 and ws.total_blocks == 11 and ws.index_rows == 22
+    assert ws.col_capacity == sum(2 * n * (n + 1) // 2 for n in N)
+    assert ws.qbar_bytes == 11 * 8 * 128 * 4 and ws.kbar_mma_bytes == 11 * 2 * 128 * 2
+    assert ws.row_ptr_bytes == 23 * 4 and ws.col_idx_bytes == ws.col_capacity * 4
+    assert ws.prefill_scratch_bytes > ws.scratch_bytes > 0
+    assert ws.scratch_bytes % 256 == 0 and ws.prefill_scratch_bytes % 256 == 0
+
+
+@pytest.mark.parametrize("kw,params,code", [
+    (dict(d=96), {}, fp2.FP2_ERR_UNSUPPORTED),
+    (dict(Hq=6, Hkv=4), {}, fp2.FP2_ERR_INVALID_ARG),
+    (dict(dtype=torch.float32), {}, fp2.FP2_ERR_UNSUPPORTED),       # f32 needs d = 64
+    (dict(dtype=torch.float8_e4m3fn, d=64), {}, fp2.FP2_ERR_UNSUPPORTED),
+    ({}, dict(block_size=32), fp2.FP2_ERR_UNSUPPORTED),
+    ({}, dict(alpha=1.5), fp2.FP2_ERR_INVALID_ARG),
+    ({}, dict(sink_blocks=-1), fp2.FP2_ERR_INVALID_ARG),
+    (dict(seqlens=(4096 * 128 + 1,)), {}, fp2.FP2_ERR_UNSUPPORTED),
+    (dict(paged=True, page_size=24), {}, fp2.FP2_ERR_UNSUPPORTED),
+])
+def test_validation_errors(kw, params, code):
+    prob = _problem(**kw)
+    p = dict(block_size=128)
+    p.update(params)
+    with pytest.raises(fp2.FP2Error) as e:
+        fp2.fp2_workspace_query(prob, fp2.make_params(**p))
+    assert e.value.status == code
+    assert fp2.fp2_last_error() != ""
+
+
+def test_chunked_prefill_rejected():
+    prob = _problem()
+    ck = np.array([0, 900, 1333], dtype=np.int32)
+    prob.struct.cu_seqlens_k_host = ck.ctypes.data_as(prob.struct.cu_seqlens_k_host.__class__)
+    with pytest.raises(fp2.FP2Error) as e:
+        fp2.fp2_workspace_query(prob, fp2.make_params(128))
+    assert e.value.status == fp2.FP2_ERR_UNSUPPORTED
+
+
+def test_scratch_too_small_rejected_before_launch():
+    prob = _problem()
+    params = fp2.make_params(128)
+    ws = fp2.fp2_workspace_query(prob, params)
+    scratch = torch.empty(ws.scratch_bytes - 256, dtype=torch.uint8)
+    pooled, _ = fp2.alloc_pooled(ws, prob, "cpu")
+    with pytest.raises(fp2.FP2Error) as e:
+        fp2.fp2_pool(prob, params, pooled, scratch, stream=0)
+    assert e.value.status == fp2.FP2_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_library_missing_fails_loudly(tmp_path):
+    with pytest.raises(FileNotFoundError):
+        fp2.load_library.__wrapped__(str(tmp_path / "nope.so")) if hasattr(fp2.load_library, "__wrapped__") \
+            else _load_fresh(str(tmp_path / "nope.so"))
+
+
+def _load_fresh(path):
+    saved = fp2._lib
+    fp2._lib = None
+    try:
+        return fp2.load_library(path)
+    finally:
+        fp2._lib = saved

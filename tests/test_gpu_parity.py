@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Small cases compare every output element and span several tiles with ragged
+tails, every supported (dtype, head_dim, block) kernel, GQA groups 1/2/4/8,
+contiguous and paged K/V (page sizes 16/64/128), varlen batches with a dense
+cutoff, alpha = 0, last-n rows, mean correction off, an external index, and
+device-side bounds checks.  The five workloads at full size compare the whole
+block index and sampled output rows.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+from synth import workloads as W
+from tests import harness as Hn
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from block_sparse_long_pooled_b200 import build
+    build.build()
+
+
+def small(name, **kw):
+    base = dict(seqlens=(1000, 333), num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=128, dtype="bf16",
+                sink_blocks=1, window_blocks=1, alpha=0.1, seed=7)
+    base.update(kw)
+    return W.Workload(name=name, **base)
+
+
+SMALL = [
+    small("bf16_g4_d128_b128", seqlens=(1000, 333)),
+    small("bf16_g8_d128_b128_paged64", num_q_heads=16, num_kv_heads=2, seqlens=(700, 1500), paged=True, page_size=64),
+    small("bf16_g1_d64_b64", num_q_heads=2, num_kv_heads=2, head_dim=64, block_size=64, seqlens=(1300,)),
+    small("bf16_g2_d64_b64_paged16", num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=64, seqlens=(500, 777),
+          paged=True, page_size=16),
+    small("bf16_g4_d64_b128", head_dim=64, seqlens=(900,)),
+    small("bf16_g4_d128_b64", block_size=64, seqlens=(1100,)),
+    small("e4m3_g4_d128_b128_paged128", dtype="e4m3", seqlens=(2000, 900), paged=True, page_size=128),
+    small("e4m3_g4_d128_b64", dtype="e4m3", block_size=64, seqlens=(1234,)),
+    small("f32_g1_d64_b64", dtype="f32", num_q_heads=1, num_kv_heads=1, head_dim=64, block_size=64, seqlens=(1024,)),
+    small("f32_g2_d64_b128", dtype="f32", num_q_heads=4, num_kv_heads=2, head_dim=64, seqlens=(640, 260)),
+    small("bf16_dense_alpha0", alpha=0.0),
+    small("bf16_no_correction", mean_correction=False, seqlens=(1500,)),
+    small("bf16_min_sparse_last_n", seqlens=(300, 1700), min_sparse_len=512, last_n_blocks=2),
+    small("bf16_tiny_and_empty_seqs", seqlens=(0, 1, 5, 130, 0, 257)),
+    small("bf16_sink2_window4", sink_blocks=2, window_blocks=4, seqlens=(2500,)),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_full_parity(w):
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    # attention on the oracle's own mask (external index) ...
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci))
+    Hn.compare_pooled(run, inp, ora)
+    stats = Hn.compare_index(run, inp, ora)
+    Hn.compare_attention_full(run, inp, ora)
+    # ... and end to end on the library's own mask
+    run2 = Hn.run_gpu(inp)
+    if stats["borderline_mismatches"] == 0:
+        Hn.compare_attention_full(run2, inp, ora)
+
+
+def test_tiny_workload_end_to_end():
+    """The 1K fp32 workload with its four planted needle blocks, through fp2_prefill."""
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    w = W.WORKLOADS["tiny_1k_f32"]
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    dev = Hn.to_device(inp)
+    prob = Hn.make_gpu_problem(inp, dev)
+    params = Hn.gpu_params(w)
+    ws = fp2.fp2_workspace_query(prob, params)
+    scratch = fp2.alloc_scratch(ws.prefill_scratch_bytes, "cuda")
+    out = torch.empty(inp.q.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty((w.num_q_heads, w.total_tokens), dtype=torch.float32, device="cuda")
+    fp2.fp2_prefill(prob, params, out, lse, scratch)
+    torch.cuda.synchronize()
+    assert fp2.fp2_get_device_status(scratch) == (0, 0)
+    # needle blocks are kept for the needle query rows' blocks
+    assert all(ora[0].kept[0, i, j] for j in inp.needle_key_blocks[0] for i in range(j, 16))
+
+    class R:
+        pass
+    run = R()
+    run.out, run.lse = out, lse
+    Hn.compare_attention_full(run, inp, ora)
+
+
+FULL = ["llama8b_32k_bf16", "llama8b_128k_bf16", "llama8b_128k_e4m3", "qwen30b_64k_paged_bf16",
+        "varlen6_paged_e4m3"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workloads(name):
+    w = W.WORKLOADS[name]
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), lse=False)
+    Hn.compare_pooled(run, inp, ora)
+    stats = Hn.compare_index(run, inp, ora)
+    print(f"{name}: density {stats['density']*100:.2f}%  borderline {stats['borderline_blocks']} "
+          f"mismatched {stats['borderline_mismatches']}")
+    Hn.compare_attention_sampled(run, inp, ora)
+    if name == "llama8b_128k_bf16":
+        assert 0.04 <= stats["density"] <= 0.06
+
+
+def test_page_table_out_of_range_is_reported_not_faulted():
+    """A corrupt page id is clamped on the device and reported through the status word."""
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    w = small("paged_corrupt", paged=True, page_size=64, seqlens=(600,))
+    inp = W.generate(w)
+    dev = Hn.to_device(inp)
+    dev["page_table"][0, 3] = 10 ** 6
+    prob = Hn.make_gpu_problem(inp, dev)
+    params = Hn.gpu_params(w)
+    ws = fp2.fp2_workspace_query(prob, params)
+    scratch = fp2.alloc_scratch(ws.prefill_scratch_bytes, "cuda")
+    out = torch.empty(inp.q.shape, dtype=torch.bfloat16, device="cuda")
+    fp2.fp2_prefill(prob, params, out, None, scratch)
+    torch.cuda.synchronize()
+    st, bits = fp2.fp2_get_device_status(scratch)
+    assert st == fp2.FP2_ERR_DEVICE_BOUNDS and bits & fp2.FP2_DEV_PAGE_OOB
+    # the context is still healthy: a clean call succeeds afterwards
+    dev["page_table"][0, 3] = int(inp.page_table[0, 3])
+    fp2.fp2_prefill(prob, params, out, None, scratch)
+    torch.cuda.synchronize()
+    assert fp2.fp2_get_device_status(scratch) == (0, 0)
+
+
+def test_external_index_without_diagonal_is_reported():
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    w = small("bad_index", seqlens=(512,))
+    inp = W.generate(w)
+    N = 4
+    rows = N * w.num_kv_heads
+    # every row keeps only block 0: rows i > 0 miss their diagonal block
+    rp = np.arange(rows + 1, dtype=np.int32)
+    ci = np.zeros(rows, dtype=np.int32)
+    dev = Hn.to_device(inp)
+    prob = Hn.make_gpu_problem(inp, dev)
+    params = Hn.gpu_params(w)
+    ws = fp2.fp2_workspace_query(prob, params)
+    pst, _ = fp2.alloc_pooled(ws, prob, "cuda")
+    scratch = fp2.alloc_scratch(ws.scratch_bytes, "cuda")
+    fp2.fp2_pool(prob, params, pst, scratch)
+    ix = fp2.index_struct(torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda())
+    out = torch.empty(inp.q.shape, dtype=torch.bfloat16, device="cuda")
+    fp2.fp2_attend(prob, params, pst, ix, out, None, scratch)
+    torch.cuda.synchronize()
+    st, bits = fp2.fp2_get_device_status(scratch)
+    assert st == fp2.FP2_ERR_DEVICE_BOUNDS and bits & fp2.FP2_DEV_INDEX_OOB
+
+
+def test_host_validation_launches_nothing():
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    w = small("val", seqlens=(256,))
+    inp = W.generate(w)
+    dev = Hn.to_device(inp)
+    prob = Hn.make_gpu_problem(inp, dev)
+    params = Hn.gpu_params(w)
+    ws = fp2.fp2_workspace_query(prob, params)
+    scratch = fp2.alloc_scratch(ws.prefill_scratch_bytes, "cuda")
+    out = torch.empty(inp.q.shape, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fp2.FP2Error) as e:
+        fp2.fp2_prefill(prob, params, out, None, scratch[: ws.prefill_scratch_bytes - 256])
+    assert e.value.status == fp2.FP2_ERR_WORKSPACE_TOO_SMALL
