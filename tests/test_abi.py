@@ -98,7 +98,9 @@ def test_scratch_too_small_rejected_before_launch():
     prob = _problem()
     params = fp2.make_params(128)
     ws = fp2.fp2_workspace_query(prob, params)
-    scratch = torch.empty(ws.scratch_bytes - 256, dtype=torch.uint8)
+    raw = torch.empty(ws.scratch_bytes + 256, dtype=torch.uint8)
+    off = (-raw.data_ptr()) % 256
+    scratch = raw[off: off + ws.scratch_bytes - 256]
     pooled, _ = fp2.alloc_pooled(ws, prob, "cpu")
     with pytest.raises(fp2.FP2Error) as e:
         fp2.fp2_pool(prob, params, pooled, scratch, stream=0)
