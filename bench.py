@@ -1,0 +1,465 @@
+"""Benchmark of mean-corrected block-sparse prefill attention (pool -> discover -> attend).
+
+One step = the whole path over one synthetic batch resident in HBM:
+fp2_pool, fp2_discover (score/threshold, scan, scatter) and fp2_attend.
+Headline metric: dense-equivalent TFLOP/s (4 d Hq sum L(L+1)/2 per step / step time);
+ms per step, achieved TFLOP/s, per-stage times, sparsity, the all-blocks-kept run of
+the same library, and an FP8 line ride along.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+Under torchrun every rank runs its own replica of the workload (the path has no
+exchange step); the time is the max over ranks and the value counts all ranks' work.
+--impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse prefill attn ms + dense-equiv & achieved TFLOPS @128K BF16/FP8, 1xB200"
+UNIT = "TFLOP/s (dense-equivalent)"
+DEFAULT_WORKLOAD = "llama8b_128k_bf16"
+FP8_WORKLOAD = "llama8b_128k_e4m3"
+
+# DRAM traffic of one attention launch on the 128K bf16 workload, from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel source it was
+# taken on (sha256 prefix of csrc/attention.cu).  None until captured.
+ATTN_TRAFFIC = {"bytes": None, "source_sha": None}
+
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks sampler
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for name, flag in zip(self.NAMES, parts[3:7]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+class Path:
+    """Device-resident inputs plus every buffer of the path for one workload."""
+
+    def __init__(self, wname, device, alpha=None):
+        import numpy as np
+        import torch
+        from block_sparse_long_pooled_b200 import fp2
+        from synth import workloads as W
+        self.fp2 = fp2
+        self.w = W.WORKLOADS[wname]
+        if alpha is not None:
+            self.w = self.w.replace(alpha=alpha)
+        w = self.w
+        inp = W.generate(w)
+        self.inp = inp
+        self.dev = device
+        self.q = inp.q.to(device)
+        if w.paged:
+            self.k, self.v = inp.k_cache.to(device), inp.v_cache.to(device)
+            self.pt = torch.from_numpy(inp.page_table).to(device)
+        else:
+            self.k, self.v, self.pt = inp.k.to(device), inp.v.to(device), None
+        self.prob = fp2.make_problem(self.q, self.k, self.v, inp.cu_seqlens, w.num_kv_heads, inp.q_descale,
+                                     inp.k_descale, inp.v_descale, page_table=self.pt)
+        self.params = fp2.make_params(w.block_size, w.alpha, w.sink_blocks, w.window_blocks, w.last_n_blocks,
+                                      w.min_sparse_len, w.mean_correction)
+        self.ws = fp2.fp2_workspace_query(self.prob, self.params)
+        self.pooled_st, self.pooled = fp2.alloc_pooled(self.ws, self.prob, device)
+        self.index_st, self.index = fp2.alloc_index(self.ws, device)
+        self.scratch = fp2.alloc_scratch(self.ws.prefill_scratch_bytes, device)
+        self.out = torch.empty(self.q.shape, dtype=fp2.out_dtype(self.prob), device=device)
+        self.np = np
+
+    def step(self, events=None):
+        f = self.fp2
+        if events:
+            events[0].record()
+        f.fp2_pool(self.prob, self.params, self.pooled_st, self.scratch)
+        if events:
+            events[1].record()
+        f.fp2_discover(self.prob, self.params, self.pooled_st, self.index_st, self.scratch)
+        if events:
+            events[2].record()
+        f.fp2_attend(self.prob, self.params, self.pooled_st, self.index_st, self.out, None, self.scratch)
+        if events:
+            events[3].record()
+
+    def work_counts(self):
+        """Kept and pruned (q head, query block, key block) tiles of the current index."""
+        np = self.np
+        w = self.w
+        rp = self.index["row_ptr"].cpu().numpy().astype(np.int64)
+        nnz_rows = np.diff(rp)
+        i_of_row = []
+        for L in w.seqlens:
+            N = -(-L // w.block_size)
+            i_of_row.append(np.repeat(np.arange(N), w.num_kv_heads))
+        i_of_row = np.concatenate(i_of_row) if i_of_row else np.zeros(0, dtype=np.int64)
+        G = w.group
+        kept = int(nnz_rows.sum()) * G
+        pruned = int(((i_of_row + 1) - nnz_rows).sum()) * G if w.mean_correction else 0
+        causal = int(sum((-(-L // w.block_size)) * (-(-L // w.block_size) + 1) // 2 for L in w.seqlens)) * \
+            w.num_q_heads
+        return kept, pruned, causal
+
+    def achieved_flops(self):
+        w = self.w
+        kept, pruned, causal = self.work_counts()
+        d, B = w.head_dim, w.block_size
+        return 4.0 * d * B * B * kept + 4.0 * d * B * pruned, kept, pruned, causal
+
+    def pool_bytes(self):
+        w = self.w
+        elt = {"f32": 4, "bf16": 2, "e4m3": 1}[w.dtype]
+        T = w.total_tokens
+        nb = self.ws.total_blocks
+        read = T * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * elt
+        write = nb * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * 4 + 2 * nb * w.num_kv_heads * w.head_dim * elt
+        return read + write
+
+
+def time_path(path, steps, warmup):
+    import torch
+    for _ in range(warmup):
+        path.step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for k in range(steps):
+        path.step(evs[k])
+    end.record()
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    st = {"pool": [], "discover": [], "attend": []}
+    for e in evs:
+        st["pool"].append(e[0].elapsed_time(e[1]))
+        st["discover"].append(e[1].elapsed_time(e[2]))
+        st["attend"].append(e[2].elapsed_time(e[3]))
+    return total, {k: sum(v) / len(v) for k, v in st.items()}
+
+
+def time_e2e(path, steps):
+    """Same path through the C ABI with host buffers: pinned H2D of Q/K/V, fp2_prefill, D2H of O."""
+    import torch
+    fp2 = path.fp2
+    hq = path.q.cpu().pin_memory()
+    hk = path.k.cpu().pin_memory()
+    hv = path.v.cpu().pin_memory()
+    hout = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+    d2h = hout.numel() * hout.element_size()
+
+    def one():
+        path.q.copy_(hq, non_blocking=True)
+        path.k.copy_(hk, non_blocking=True)
+        path.v.copy_(hv, non_blocking=True)
+        fp2.fp2_prefill(path.prob, path.params, path.out, None, path.scratch)
+        hout.copy_(path.out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps, h2d, d2h
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+
+class OracleSampler:
+    """The fp64 oracle on a bounded sample of a workload (generated once).
+
+    A sample pools every block and runs discovery for every KV-head group of the
+    longest sequence, then times exact + mean-corrected attention for n uniformly
+    drawn (group, query block) pairs (all G heads, all tokens of the block).  The
+    full-workload time is estimated as discovery time + mean pair time x pairs,
+    scaled by total tokens / sampled sequence tokens for varlen batches."""
+
+    def __init__(self, wname):
+        import numpy as np
+        from oracle import fp2_oracle as O
+        from synth import workloads as W
+        self.O, self.np = O, np
+        self.w = w = W.WORKLOADS[wname]
+        self.inp = W.generate(w)
+        self.r = int(np.argmax(w.seqlens))
+        self.p = O.SparseParams(block_size=w.block_size, alpha=w.alpha, sink_blocks=w.sink_blocks,
+                                window_blocks=w.window_blocks, last_n_blocks=w.last_n_blocks,
+                                min_sparse_len=w.min_sparse_len, mean_correction=w.mean_correction)
+
+    def _group_inputs(self, g):
+        O, inp, w = self.O, self.inp, self.w
+        a, b = int(inp.cu_seqlens[self.r]), int(inp.cu_seqlens[self.r + 1])
+        L = b - a
+        heads = list(range(g * w.group, (g + 1) * w.group))
+        q = inp.dequant("q", heads=heads, tokens=slice(a, b))
+        if w.paged:
+            import torch
+            kc = inp.k_cache[:, :, g:g + 1].to(torch.float64).numpy() * inp.k_descale
+            vc = inp.v_cache[:, :, g:g + 1].to(torch.float64).numpy() * inp.v_descale
+            k = O.gather_paged(kc, inp.page_table[self.r:self.r + 1], [L])
+            v = O.gather_paged(vc, inp.page_table[self.r:self.r + 1], [L])
+        else:
+            k = inp.dequant("k", heads=[g], tokens=slice(a, b))
+            v = inp.dequant("v", heads=[g], tokens=slice(a, b))
+        return q, k, v, L
+
+    def run(self, n_pairs, seed=0):
+        O, np, w = self.O, self.np, self.w
+        B, G = w.block_size, w.group
+        scale = 1.0 / math.sqrt(w.head_dim)
+        rng = np.random.default_rng(seed)
+        L = w.seqlens[self.r]
+        N = -(-L // B)
+        pairs = rng.integers(0, w.num_kv_heads * N, size=n_pairs)
+        t_disc = t_attn = 0.0
+        for g in range(w.num_kv_heads):
+            q, k, v, L = self._group_inputs(g)
+            t0 = time.perf_counter()
+            qbar, counts = O.pool_blocks(q, B)
+            kbar, _ = O.pool_blocks(k, B)
+            vbar, _ = O.pool_blocks(v, B)
+            kept, _ = O.select_blocks(O.block_scores(qbar, kbar, scale), 1, L, self.p)
+            t1 = time.perf_counter()
+            t_disc += t1 - t0
+            for pr in pairs[pairs // N == g]:
+                i = int(pr % N)
+                rows = np.array([[t, h] for t in range(i * B, min(L, (i + 1) * B)) for h in range(G)])
+                t2 = time.perf_counter()
+                O.attend(q, k, v, kbar, vbar, counts, kept, B, scale, w.mean_correction, rows=rows)
+                t_attn += time.perf_counter() - t2
+        est = (t_disc + t_attn / max(1, n_pairs) * w.num_kv_heads * N) * (w.total_tokens / L)
+        desc = (f"fp64 oracle: pooling + discovery of all {w.num_kv_heads} KV-head groups of the {L}-token "
+                f"sequence, attention for {n_pairs} uniformly drawn (group, query block) pairs of "
+                f"{w.num_kv_heads * N}; full time = discovery + mean pair time x pairs")
+        return t_disc + t_attn, est, desc
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def run_reference(args, rank, world):
+    from synth import workloads as W
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    dense = w.dense_equiv_flops()
+    sampler = OracleSampler(args.workload)
+    for k in range(args.warmup):
+        sampler.run(2, seed=1000 + k)
+    times, ests, desc = [], [], ""
+    for k in range(args.steps):
+        t, est, desc = sampler.run(4, seed=k)
+        times.append(t)
+        ests.append(est)
+    est = statistics.mean(ests)
+    value = dense / est / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": max(w.seqlens), "heads": f"{w.num_q_heads}/{w.num_kv_heads}",
+                       "head_dim": w.head_dim, "block": w.block_size, "parallelism": f"replicas{args.gpus}"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc + f"; mean over {args.steps} samples of {statistics.mean(times):.1f} s"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-extras", action="store_true", help="skip the FP8, all-kept, e2e and CPU legs")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    from block_sparse_long_pooled_b200 import build, fp2
+    build.build()
+    fp2.load_library()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        pg = dist
+    peaks = load_peaks()
+
+    path = Path(args.workload, dev)
+    w = path.w
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    total_ms, stages = time_path(path, args.steps, args.warmup)
+    clocks = sampler.stop()
+    if pg:
+        t = torch.tensor([total_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+        pg.barrier()
+    st, bits = fp2.fp2_get_device_status(path.scratch)
+    if st != fp2.FP2_OK:
+        raise SystemExit(f"device status {bits:#x}")
+    ms = total_ms / args.steps
+    dense = w.dense_equiv_flops()
+    ach, kept, pruned, causal = path.achieved_flops()
+    value = dense * world / (ms * 1e-3) / 1e12
+    attn_tflops = ach / (stages["attend"] * 1e-3) / 1e12
+    peak_bf16 = peaks["bf16_tflops_sustained"]
+    peak = peak_bf16 if w.dtype != "e4m3" else 2.0 * peak_bf16
+    sha = source_sha(os.path.join(ROOT, "block_sparse_long_pooled_b200", "csrc", "attention.cu"))
+    traffic = ATTN_TRAFFIC["bytes"] if ATTN_TRAFFIC["source_sha"] == sha else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded NIAH-style generator, see DESIGN.md)",
+        "config": {"workload": w.name, "seq_len": max(w.seqlens), "batch": len(w.seqlens),
+                   "heads": f"{w.num_q_heads}/{w.num_kv_heads}", "head_dim": w.head_dim, "block": w.block_size,
+                   "alpha": w.alpha, "sink": w.sink_blocks, "window": w.window_blocks,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2 ({(path.q.numel() * path.q.element_size() + 2 * path.k.numel() * path.k.element_size()) / 1e9:.2f} GB)"},
+        "achieved_tflops": ach / (ms * 1e-3) / 1e12,
+        "sparsity": kept / causal,
+        "stages_ms": stages,
+        "roofline": {"kernel": "attention_kernel", "bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16 sustained" + (" x2 (FP8 nominal ratio)" if w.dtype == "e4m3" else "")},
+        "pool_roofline": {"bound": "hbm", "achieved": path.pool_bytes() / (stages["pool"] * 1e-3) / 1e9,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": path.pool_bytes() / (stages["pool"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "clocks": clocks,
+        "gpu_launches": 5 * args.steps,
+    }
+    if not args.no_extras:
+        # the same library with every block kept (alpha = 0) on the same inputs
+        dense_path = Path(args.workload, dev, alpha=0.0)
+        dms, dst = time_path(dense_path, max(3, args.steps // 8), 2)
+        dach, _, _, _ = dense_path.achieved_flops()
+        line["all_kept"] = {"ms_per_step": dms / max(3, args.steps // 8),
+                            "attend_tflops": dach / (dst["attend"] * 1e-3) / 1e12,
+                            "attend_frac": dach / (dst["attend"] * 1e-3) / 1e12 / peak}
+        del dense_path
+        e2e_ms, h2d, d2h = time_e2e(path, max(3, args.steps // 8))
+        line["e2e"] = {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        if args.workload == DEFAULT_WORKLOAD:
+            del path
+            torch.cuda.empty_cache()
+            p8 = Path(FP8_WORKLOAD, dev)
+            ms8, st8 = time_path(p8, args.steps, args.warmup)
+            a8, k8, _, c8 = p8.achieved_flops()
+            t8 = a8 / (st8["attend"] * 1e-3) / 1e12
+            line["fp8"] = {"workload": FP8_WORKLOAD, "ms_per_step": ms8 / args.steps,
+                           "value": p8.w.dense_equiv_flops() / (ms8 / args.steps * 1e-3) / 1e12,
+                           "achieved_tflops": a8 / (ms8 / args.steps * 1e-3) / 1e12, "sparsity": k8 / c8,
+                           "stages_ms": st8, "attend_tflops": t8, "attend_frac_of_fp8_peak": t8 / (2 * peak_bf16),
+                           "attend_frac_of_bf16_peak": t8 / peak_bf16}
+            del p8
+        if rank == 0 and world == 1:
+            secs, est, desc = OracleSampler(args.workload).run(400)
+            line["cpu_baseline"] = {"value": dense / est / 1e12, "unit": UNIT, "cores": cpu_cores(),
+                                    "kind": "oracle", "sample": desc + f" ({secs:.1f} s of CPU work)"}
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

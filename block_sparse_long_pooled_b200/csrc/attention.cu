@@ -16,8 +16,8 @@
 // Warp roles (320 threads):
 //   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S,
 //                    mask, online max with lazy O rescale (only when the running max grows
-//                    by more than 2^8), write P (bf16 / e4m3 / f32) back over S in TMEM,
-//                    and finally normalise O and store it.
+//                    past a threshold), write P (bf16, f32, or e4m3 as a hi + lo pair of
+//                    planes) back over S in TMEM, and finally normalise O and store it.
 //   warp 8           producer: builds the kept-block bitmask, issues TMA loads of Q once and
 //                    of K/V (or kbar/vbar) tiles into an NSLOT ring of shared-memory slots.
 //   warp 9           MMA issuer (one thread): S_s = Q_s K^T (SS form) and O_s += P_s V (A
@@ -47,6 +47,12 @@ struct AttnCfg {
   static constexpr int S_COL0 = 0, S_COL1 = BN;
   static constexpr int O_COL0 = 2 * BN, O_COL1 = 2 * BN + D;
   static constexpr int TMEM_COLS = 512;
+  // Online-softmax constants (log2 domain).  P is written as 2^(x - m + P_SHIFT); the running
+  // max m is only raised when the row max grows by more than LAZY, so P <= 2^(P_SHIFT + LAZY).
+  // e4m3: P_SHIFT 4 keeps small probabilities out of e4m3's subnormal range and 2^8 stays
+  // below its 448 maximum; P is then sent as two e4m3 terms (hi + lo).
+  static constexpr float P_SHIFT = DT == 2 ? 4.0f : 0.0f;
+  static constexpr float LAZY = DT == 2 ? 4.0f : 8.0f;
   static constexpr uint32_t IDESC_S = make_idesc(FMT, FMT, 0, 0, 128, BN);
   static constexpr uint32_t IDESC_PV = make_idesc(FMT, FMT, 0, 1, 128, D);
   static constexpr int OFF_Q = 0;
@@ -301,7 +307,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int k = 0; k < BN / C::UK; ++k) {
             const uint64_t bd = smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
-            umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+            if constexpr (DT == 2) {
+              umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+              umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
+            } else {
+              umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+            }
           }
           umma_commit(&o_done[s]);
         }
@@ -348,7 +359,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       const float m_new = fmaxf(m_run, mt);
-      const bool need = m_new > m_run + 8.0f;
+      const bool need = m_new > m_run + C::LAZY;
       if (jt > 0 && __any_sync(0xFFFFFFFFu, need)) {
         const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll
@@ -365,7 +376,7 @@ __global__ void __launch_bounds__(320, 1)
         l_run = (m_run == -CUDART_INF_F) ? 0.f : l_run * fast_exp2(m_run - m_new);
         m_run = m_new;
       }
-      const float mu = (m_run == -CUDART_INF_F) ? 0.f : m_run;
+      const float mu = ((m_run == -CUDART_INF_F) ? 0.f : m_run) - C::P_SHIFT;
       // Pass 2: P = 2^(x - m), packed to the MMA type and written over the columns of S
       // already consumed (chunk c of P lands at or before chunk c of S).
       float rsum = 0.f;
@@ -386,10 +397,12 @@ __global__ void __launch_bounds__(320, 1)
           for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
           tmem_st16(s_addr + c * 16, pk);
         } else if constexpr (DT == 2) {
-          uint32_t pk[8];
+          // K-step c of the PV MMA: hi plane at columns [16c, 16c+8), lo plane at [16c+8, 16c+16).
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) pk[e] = pack_e4m3x4(pv[4 * e], pv[4 * e + 1], pv[4 * e + 2], pv[4 * e + 3]);
-          tmem_st8(s_addr + c * 8, pk);
+          for (int e = 0; e < 8; ++e)
+            split_e4m3x4(pv[4 * e], pv[4 * e + 1], pv[4 * e + 2], pv[4 * e + 3], pk[e], pk[8 + e]);
+          tmem_st16(s_addr + c * 16, pk);
         } else {
           uint32_t pk[32];
 #pragma unroll
@@ -437,7 +450,8 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       if (row_ok && a.lse != nullptr)
-        a.lse[static_cast<int64_t>(h) * a.total_tokens + tok] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+        a.lse[static_cast<int64_t>(h) * a.total_tokens + tok] =
+            (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f;
     }
   }
 
