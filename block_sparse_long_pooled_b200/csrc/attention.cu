@@ -306,7 +306,10 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
 #pragma unroll
           for (int k = 0; k < BN / C::UK; ++k) {
-            const uint64_t bd = smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
+            // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with
+            // 4-row atoms (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
+            const uint64_t bd = DT == 0 ? smem_desc(vaddr + k * C::UK * 128, BN * 128, 512, 1u)
+                                        : smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
             if constexpr (DT == 2) {
               umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
               umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);

@@ -177,8 +177,10 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // 3-D map over a token-major tensor: dims {d, heads, rows}, box {128B/elt, 1, box_rows}, 128B swizzle.
+// mn_major_32b: the tile feeds the MMA as an MN-major 32-bit operand (f32 V), which needs the
+// 32-byte-chunk flavour of the 128-byte swizzle.
 fp2_status encode_3d(CUtensorMap* m, fp2_dtype dt, const void* base, int D, int heads, int64_t rows,
-                     int64_t row_stride_elems, int box_rows) {
+                     int64_t row_stride_elems, int box_rows, bool mn_major_32b = false) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return fail(FP2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   const int elt = elt_bytes(dt);
@@ -191,7 +193,8 @@ fp2_status encode_3d(CUtensorMap* m, fp2_dtype dt, const void* base, int D, int 
   const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elt), 1u, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = fn(m, t, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        mn_major_32b ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FP2_ERR_CUDA, "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(r));
   return FP2_OK;
@@ -305,12 +308,13 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   const int kv_box = paged ? std::min(B, p->page_size) : B;
   if ((st2 = encode_3d(&a.tm_k, p->dtype, p->k, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box)) != FP2_OK)
     return st2;
-  if ((st2 = encode_3d(&a.tm_v, p->dtype, p->v, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box)) != FP2_OK)
+  const bool v32 = p->dtype == FP2_F32;
+  if ((st2 = encode_3d(&a.tm_v, p->dtype, p->v, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box, v32)) != FP2_OK)
     return st2;
   const int64_t hd = static_cast<int64_t>(p->num_kv_heads) * D;
   if ((st2 = encode_3d(&a.tm_kb, p->dtype, pl->kbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B)) != FP2_OK)
     return st2;
-  if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B)) != FP2_OK)
+  if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B, v32)) != FP2_OK)
     return st2;
   a.row_ptr = ix->row_ptr;
   a.col_idx = ix->col_idx;

@@ -126,17 +126,19 @@ FP2_DEVICE void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 FP2_DEVICE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 FP2_DEVICE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Shared-memory matrix descriptor, 128-byte swizzle (sm100 encoding: version 1 at bit 46,
-// layout type 2 at bits 61-63).  lbo/sbo in bytes.
-FP2_DEVICE uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor (sm100 encoding: version 1 at bit 46, layout type at bits
+// 61-63: 2 = 128-byte swizzle of 16-byte chunks, 1 = 128-byte swizzle of 32-byte chunks, the
+// only layout the tensor cores accept for MN-major 32-bit operands).  lbo/sbo in bytes.
+FP2_DEVICE uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
   d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;
-  d |= 2ull << 61;
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
 }
+FP2_DEVICE uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) { return smem_desc(saddr, lbo, sbo, 2u); }
 
 // Instruction descriptor: f32 accumulator, operand formats, majors, N and M.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_mn_major,

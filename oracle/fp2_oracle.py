@@ -157,6 +157,9 @@ def select_blocks(s: np.ndarray, num_kv_heads: int, L: int, p: SparseParams):
     """
     Hq, N, _ = s.shape
     G = Hq // num_kv_heads
+    if N == 0:
+        empty = np.zeros((num_kv_heads, 0, 0), dtype=bool)
+        return empty, empty.copy()
     forced = forced_blocks(N, L, p)
     causal = np.tri(N, dtype=bool)
     kept = np.zeros((num_kv_heads, N, N), dtype=bool)

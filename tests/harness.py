@@ -21,6 +21,12 @@ from oracle import fp2_oracle as O
 from synth import workloads as W
 
 TOL = {"bf16": (2e-2, 5e-3), "f32": (2e-2, 5e-3), "e4m3": (6e-2, 2e-2)}
+# LSE (natural log) bounds.  bf16: inputs are exact bf16; rounding kbar to bf16 moves a pruned
+# block's logit q.kbar*scale by <= 2^-9 of it (<= 2e-2 for pooled logits up to ~10).  e4m3: kbar
+# rounded to e4m3 moves it by <= 2^-4 of q.kbar*scale (pooled logits <= ~2 -> 1.5e-1).  f32: the
+# tf32 tensor cores keep 10 mantissa bits of fp32 Q and K, so a logit q.k*scale moves by up to
+# ~2^-10 of sum|q_i k_i|*scale; needle pairs reach 9*sqrt(d) = 72 at d = 64 -> 1e-1.
+LSE_TOL = {"bf16": 2e-2, "f32": 1e-1, "e4m3": 1.5e-1}
 
 
 def oracle_params(w: W.Workload) -> O.SparseParams:
@@ -251,7 +257,7 @@ def compare_attention_full(run: GpuRun, inp: W.Inputs, ora: list, kept_override:
     if run.lse is not None:
         lse = run.lse.cpu().numpy().astype(np.float64)
         lse_ref = np.concatenate(L_ref, axis=1)
-        assert float(np.abs(lse - lse_ref).max()) < 5e-2, float(np.abs(lse - lse_ref).max())
+        assert float(np.abs(lse - lse_ref).max()) < LSE_TOL[w.dtype], float(np.abs(lse - lse_ref).max())
     return maxabs, rel
 
 
