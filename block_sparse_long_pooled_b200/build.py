@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp2.so")
-SOURCES = ["fp2_api.cu", "pool.cu", "discover.cu", "attention.cu"]
+SOURCES = ["fp2_api.cu", "pool.cu", "discover.cu", "attention.cu", "fp2_noalloc.cu"]
 HEADERS = ["fp2_device.cuh", "fp2_kernels.h", "fp2_plan.h", os.path.join("..", "..", "include", "fp2.h")]
 
 

@@ -350,6 +350,35 @@ fp2_status clear_status(void* scratch, cudaStream_t st) {
 
 }  // namespace
 
+// Used by fp2_noalloc.cu only: discovery into a caller-supplied scratch region of a fixed capacity,
+// optionally copying the device status word to status_dev afterwards.
+namespace fp2_internal {
+
+fp2_status set_error(fp2_status s, const char* msg) { return fail(s, msg); }
+
+fp2_status discover_fixed_scratch(const fp2_problem* problem, const fp2_sparse_params* params,
+                                  const fp2_pooled* pooled, const fp2_index* index, void* scratch,
+                                  size_t capacity, uint32_t* status_dev, cudaStream_t st) {
+  Ctx c;
+  fp2_status s;
+  if ((s = validate(problem, params, c)) != FP2_OK) return s;
+  if (c.ws.scratch_bytes > capacity)
+    return fail(FP2_ERR_UNSUPPORTED, "problem needs " + std::to_string(c.ws.scratch_bytes) +
+                                         " bytes of discovery scratch; the static buffer holds " +
+                                         std::to_string(capacity));
+  if ((s = check_pooled(pooled, true)) != FP2_OK) return s;
+  if ((s = check_index(index, c)) != FP2_OK) return s;
+  if ((s = clear_status(scratch, st)) != FP2_OK) return s;
+  if (c.T > 0 && (s = run_discover(problem, params, c, pooled, index, scratch, st)) != FP2_OK) return s;
+  if (status_dev != nullptr) {
+    const cudaError_t e = cudaMemcpyAsync(status_dev, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "status copy");
+  }
+  return FP2_OK;
+}
+
+}  // namespace fp2_internal
+
 extern "C" {
 
 fp2_status fp2_workspace_query(const fp2_problem* problem, const fp2_sparse_params* params, fp2_workspace* out) {

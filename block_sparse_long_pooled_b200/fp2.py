@@ -27,7 +27,8 @@ STATUS_NAMES = {0: "FP2_OK", 1: "FP2_ERR_INVALID_ARG", 2: "FP2_ERR_UNSUPPORTED",
                 4: "FP2_ERR_CUDA", 5: "FP2_ERR_DEVICE_BOUNDS", 6: "FP2_ERR_TIMEOUT"}
 
 EXPORTED = ("fp2_workspace_query", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
-            "fp2_get_device_status", "fp2_last_error", "fp2_version")
+            "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static")
+FP2_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class fp2_problem(ctypes.Structure):
@@ -99,8 +100,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp2_attend.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_pooled), P(fp2_index), vp, vp, vp, sz, vp]
     lib.fp2_prefill.argtypes = [P(fp2_problem), P(fp2_sparse_params), vp, vp, vp, sz, vp]
     lib.fp2_get_device_status.argtypes = [vp, P(ctypes.c_uint32)]
+    lib.fp2_discover_static.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_pooled), P(fp2_index), vp, vp]
     for name in ("fp2_workspace_query", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
-                 "fp2_get_device_status"):
+                 "fp2_get_device_status", "fp2_discover_static"):
         getattr(lib, name).restype = ctypes.c_int
     lib.fp2_last_error.argtypes = []
     lib.fp2_last_error.restype = ctypes.c_char_p
@@ -207,6 +209,17 @@ def fp2_prefill(problem: Problem, params, out, lse, scratch, stream=None):
     _check(load_library().fp2_prefill(ctypes.byref(problem.struct), ctypes.byref(params), _ptr(out), _ptr(lse),
                                       _ptr(scratch), scratch.numel() * scratch.element_size(),
                                       _stream_handle(stream)))
+
+
+def fp2_discover_static(problem: Problem, params, pooled: fp2_pooled, index: fp2_index, status_dev=None,
+                        stream=None):
+    """fp2_discover without a scratch argument, for callers that cannot allocate device memory where
+    they run discovery.  The library keeps the scratch in its own static device buffer (shared by all
+    calls on a GPU: do not overlap calls).  status_dev: optional int32/uint32 device tensor of >= 1
+    element that receives the call's FP2_DEV_* status word."""
+    _check(load_library().fp2_discover_static(ctypes.byref(problem.struct), ctypes.byref(params),
+                                              ctypes.byref(pooled), ctypes.byref(index), _ptr(status_dev),
+                                              _stream_handle(stream)))
 
 
 def fp2_get_device_status(scratch) -> tuple:

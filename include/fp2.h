@@ -179,6 +179,22 @@ FP2_API fp2_status fp2_prefill(const fp2_problem* problem, const fp2_sparse_para
  * return value maps them to FP2_ERR_DEVICE_BOUNDS / FP2_ERR_TIMEOUT, else FP2_OK. */
 FP2_API fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_out);
 
+/* Size of the device buffer fp2_discover_static uses in place of caller scratch. */
+#define FP2_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* Discovery for callers that cannot allocate device memory where they run it (a serving runtime
+ * that reserved all memory up front and forbids allocation on the request path, or a C host with no
+ * device allocator).  The paper has no counterpart: this is fp2_discover with its scratch moved into
+ * a library-owned static __device__ buffer of FP2_STATIC_SCRATCH_BYTES per GPU, held until exit.
+ * Inputs (pooled) and outputs (index) are still the caller's.  Returns FP2_ERR_UNSUPPORTED when the
+ * problem's fp2_workspace.scratch_bytes exceeds FP2_STATIC_SCRATCH_BYTES.  Allocates nothing.  The
+ * first call on a device looks up the buffer's address (make it before any stream capture).  All
+ * calls share the buffer: calls that overlap on the GPU race, so serialise them.  status_dev
+ * (device pointer, or NULL) receives a copy of the FP2_DEV_* status word of this call. */
+FP2_API fp2_status fp2_discover_static(const fp2_problem* problem, const fp2_sparse_params* params,
+                                       const fp2_pooled* pooled, const fp2_index* index, uint32_t* status_dev,
+                                       fp2_stream_t stream);
+
 /* Message for the last failing call on this thread ("" if none). */
 FP2_API const char* fp2_last_error(void);
 
