@@ -13,7 +13,7 @@
 // correction shares the exact path's MMAs and online softmax; kept blocks and blocks >= i
 // are masked out of the virtual tiles.  The last kept block is the diagonal (causal mask).
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S,
 //                    mask, online max with lazy O rescale (only when the running max grows
 //                    past a threshold), write P (bf16, f32, or e4m3 as a hi + lo pair of
@@ -22,6 +22,7 @@
 //                    of K/V (or kbar/vbar) tiles into an NSLOT ring of shared-memory slots.
 //   warp 9           MMA issuer (one thread): S_s = Q_s K^T (SS form) and O_s += P_s V (A
 //                    operand P read from TMEM), tcgen05.commit to mbarriers.
+//   warps 10-11      idle (they complete warpgroup 2 for the register split).
 // TMEM: S0 | S1 | O0 | O1 (512 columns); P_s aliases S_s.
 #include <math_constants.h>
 
@@ -29,6 +30,10 @@
 #include "fp2_kernels.h"
 
 namespace fp2 {
+
+#ifndef REG_LOW_T
+#define REG_LOW_T 56
+#endif
 
 template <int DT, int D, int BN>
 struct AttnCfg {
@@ -47,6 +52,10 @@ struct AttnCfg {
   static constexpr int S_COL0 = 0, S_COL1 = BN;
   static constexpr int O_COL0 = 2 * BN, O_COL1 = 2 * BN + D;
   static constexpr int TMEM_COLS = 512;
+  static constexpr int REG_LOW = REG_LOW_T;
+  static constexpr int REG_HIGH = ((384 * 168 - 128 * REG_LOW) / 256) / 8 * 8 > 248
+                                      ? 248 : ((384 * 168 - 128 * REG_LOW) / 256) / 8 * 8;
+  static_assert(128 * REG_LOW + 256 * REG_HIGH <= 384 * 168, "register split exceeds the launch");
   // Online-softmax constants (log2 domain).  P is written as 2^(x - m + P_SHIFT); the running
   // max m is only raised when the row max grows by more than LAZY, so P <= 2^(P_SHIFT + LAZY).
   // e4m3: P_SHIFT 4 keeps small probabilities out of e4m3's subnormal range and 2^8 stays
@@ -86,6 +95,32 @@ FP2_DEVICE void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
+// tcgen05.ld of 64 consecutive columns (2 x 32) followed by its wait, in one statement so
+// that no use of the registers can be scheduled before the data has landed.
+FP2_DEVICE void tmem_ld64_sync(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr + 0u), "r"(taddr + 32u)
+      : "memory");
+}
+
+// tcgen05.ld of 128 consecutive columns (4 x 32) followed by its wait, in one statement so
+// that no use of the registers can be scheduled before the data has landed.
+FP2_DEVICE void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr + 0u), "r"(taddr + 32u), "r"(taddr + 64u), "r"(taddr + 96u)
+      : "memory");
+}
+
 // Bit e of the result is set when pooled block (base + e) is a pruned block of query block i:
 // strictly left of the diagonal and absent from the kept set.
 FP2_DEVICE uint32_t pruned_word(const uint32_t* kmask, int base, int i) {
@@ -94,15 +129,6 @@ FP2_DEVICE uint32_t pruned_word(const uint32_t* kmask, int base, int i) {
   const int nvalid = i - base;  // blocks base .. i-1 are candidates
   const uint32_t lim = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
   return ~kept & lim;
-}
-
-// Scaled logit (log2 domain) of one S element with the tile's mask applied.
-FP2_DEVICE float logit(uint32_t sbits, float scale_log2, bool virt, bool diag, uint32_t mword, int e, int col,
-                       int tl, float log2_blk) {
-  const float xv = __uint_as_float(sbits) * scale_log2;
-  if (virt) return ((mword >> e) & 1u) ? xv + log2_blk : -CUDART_INF_F;
-  if (diag && col > tl) return -CUDART_INF_F;
-  return xv;
 }
 
 // Bounded wait used only while draining in-flight copies at exit; ignores the abort flag.
@@ -118,7 +144,7 @@ FP2_DEVICE void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status
 }
 
 template <int DT, int D, int BN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attention_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ Fp2Plan P) {
   using C = AttnCfg<DT, D, BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -177,284 +203,327 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Register split: the launch gives 384 threads x 168 registers; warpgroup 2 (producer, MMA,
+  // two idle warps) drops to 56 and the two softmax warpgroups rise to 224:
+  // 128 x 56 + 256 x 224 = 64512 = 384 x 168.
+  // Register split: the launch gives 384 threads x 168 registers; warpgroup 2 (producer, MMA,
+  // two idle warps) drops to REG_LOW and the two softmax warpgroups rise to REG_HIGH, with
+  // 128 * REG_LOW + 256 * REG_HIGH <= 384 * 168 (checked at compile time).
 
-  if (warp == 8) {
-    // ---------------------------------------------------------------- producer
-    const int nw = (i + 32) / 32;
-    for (int w = lane; w < nw; w += 32) kmask[w] = 0u;
-    __syncwarp();
-    bool bad = false;
-    for (int e = lane; e < nkept; e += 32) {
-      const int j = a.col_idx[rs + e];
-      const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
-      if (j < 0 || j > i || j <= prev)
-        bad = true;
-      else
-        atomicOr(&kmask[j >> 5], 1u << (j & 31));
-    }
-    if (lane == 0 && a.col_idx[re - 1] != i) bad = true;
-    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
-    __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(mask_ready);
-      tma_prefetch_desc(&a.tm_q);
-      tma_prefetch_desc(&a.tm_k);
-      tma_prefetch_desc(&a.tm_v);
-      tma_prefetch_desc(&a.tm_kb);
-      tma_prefetch_desc(&a.tm_vb);
-      constexpr int HS = 128 / BN;
-      const int tokq = P.tok_off[r] + i * BN;
-      for (int s = 0; s < a.NT; ++s) {
-        mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
-        for (int hs = 0; hs < HS; ++hs) {
-          const int hl = (part * a.NT + s) * HS + hs;
-          const int h = g * a.G + (hl % a.G);
-          for (int c = 0; c < C::DCH; ++c)
-            tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + c * (128 * 128) + hs * (BN * 128), &a.tm_q, &q_full[s],
-                        c * C::KCH, h, tokq);
-        }
+  if (warp >= 8) {
+    setmaxnreg_dec<C::REG_LOW>();
+    if (warp == 8) {
+      // ---------------------------------------------------------------- producer
+      const int nw = (i + 32) / 32;
+      for (int w = lane; w < nw; w += 32) kmask[w] = 0u;
+      __syncwarp();
+      bool bad = false;
+      for (int e = lane; e < nkept; e += 32) {
+        const int j = a.col_idx[rs + e];
+        const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
+        if (j < 0 || j > i || j <= prev)
+          bad = true;
+        else
+          atomicOr(&kmask[j >> 5], 1u << (j & 31));
       }
-      int p = 0;
-      for (int jt = 0; jt < n_tiles && !*abort_flag; ++jt) {
-        int j = -1;
-        if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), i);
-        bool stop = false;
-        for (int kv = 0; kv < 2; ++kv) {
-          const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
-          if (wrap > 0 && !mbar_wait(&kv_empty[slot], (wrap - 1) & 1, abort_flag, a.status)) {
-            stop = true;
-            break;
+      if (lane == 0 && a.col_idx[re - 1] != i) bad = true;
+      if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(mask_ready);
+        tma_prefetch_desc(&a.tm_q);
+        tma_prefetch_desc(&a.tm_k);
+        tma_prefetch_desc(&a.tm_v);
+        tma_prefetch_desc(&a.tm_kb);
+        tma_prefetch_desc(&a.tm_vb);
+        constexpr int HS = 128 / BN;
+        const int tokq = P.tok_off[r] + i * BN;
+        for (int s = 0; s < a.NT; ++s) {
+          mbar_arrive_expect_tx(&q_full[s], C::Q_BYTES);
+          for (int hs = 0; hs < HS; ++hs) {
+            const int hl = (part * a.NT + s) * HS + hs;
+            const int h = g * a.G + (hl % a.G);
+            for (int c = 0; c < C::DCH; ++c)
+              tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + c * (128 * 128) + hs * (BN * 128), &a.tm_q, &q_full[s],
+                          c * C::KCH, h, tokq);
           }
-          mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
-          uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
-          if (j < 0) {
-            const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
-            for (int c = 0; c < C::DCH; ++c)
-              tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.blk_off[r] + jt * BN);
-          } else if (a.page_table == nullptr) {
-            const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
-            for (int c = 0; c < C::DCH; ++c)
-              tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.tok_off[r] + j * BN);
-          } else {
-            const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
-            const int PR = min(BN, a.page_size);
-            for (int sb = 0; sb < BN / PR; ++sb) {
-              int t = j * BN + sb * PR;
-              if (t >= L) t = (L - 1) - ((L - 1) % PR);  // past the end: reload the last rows (masked)
-              int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + t / a.page_size];
-              if (page < 0 || page >= a.num_pages) {
-                set_status(a.status, FP2_DEV_PAGE_OOB);
-                page = 0;
-              }
-              const int flat = page * a.page_size + (t % a.page_size);
-              for (int c = 0; c < C::DCH; ++c)
-                tma_load_3d(dst + c * (BN * 128) + sb * (PR * 128), tm, &kv_full[slot], c * C::KCH, g, flat);
+        }
+        int p = 0;
+        for (int jt = 0; jt < n_tiles && !*abort_flag; ++jt) {
+          int j = -1;
+          if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), i);
+          bool stop = false;
+          for (int kv = 0; kv < 2; ++kv) {
+            const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
+            if (wrap > 0 && !mbar_wait(&kv_empty[slot], (wrap - 1) & 1, abort_flag, a.status)) {
+              stop = true;
+              break;
             }
+            mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
+            uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
+            if (j < 0) {
+              const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
+              for (int c = 0; c < C::DCH; ++c)
+                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.blk_off[r] + jt * BN);
+            } else if (a.page_table == nullptr) {
+              const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
+              for (int c = 0; c < C::DCH; ++c)
+                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.tok_off[r] + j * BN);
+            } else {
+              const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
+              const int PR = min(BN, a.page_size);
+              for (int sb = 0; sb < BN / PR; ++sb) {
+                int t = j * BN + sb * PR;
+                if (t >= L) t = (L - 1) - ((L - 1) % PR);  // past the end: reload the last rows (masked)
+                int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + t / a.page_size];
+                if (page < 0 || page >= a.num_pages) {
+                  set_status(a.status, FP2_DEV_PAGE_OOB);
+                  page = 0;
+                }
+                const int flat = page * a.page_size + (t % a.page_size);
+                for (int c = 0; c < C::DCH; ++c)
+                  tma_load_3d(dst + c * (BN * 128) + sb * (PR * 128), tm, &kv_full[slot], c * C::KCH, g, flat);
+              }
+            }
+            ++p;
           }
+          if (stop) break;
+        }
+        // Never leave with copies in flight.
+        for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status);
+        for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status);
+      }
+    } else if (warp == 9) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        bool ok = true;
+        for (int s = 0; s < a.NT && ok; ++s) ok = mbar_wait(&q_full[s], 0, abort_flag, a.status);
+        tc_fence_after();
+        int p = 0;
+        for (int jt = 0; jt < n_tiles && ok; ++jt) {
+          int slot = p % C::NSLOT;
+          if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
+          tc_fence_after();
+          const uint32_t kaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
+          for (int s = 0; s < a.NT; ++s) {
+            if (jt > 0 && !mbar_wait(&o_done[s], (jt - 1) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t qaddr = sbase + C::OFF_Q + s * C::Q_BYTES;
+            const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+  #pragma unroll
+            for (int k = 0; k < D / C::UK; ++k) {
+              const int c = (k * C::UK) / C::KCH;
+              const int koff = ((k * C::UK) % C::KCH) * C::ELT;
+              const uint64_t ad = smem_desc_sw128(qaddr + c * (128 * 128) + koff, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(kaddr + c * (BN * 128) + koff, 16, 1024);
+              umma_ss<C::KIND>(dcol, ad, bd, C::IDESC_S, k > 0 ? 1u : 0u);
+            }
+            umma_commit(&s_full[s]);
+          }
+          if (!ok) break;
+          umma_commit(&kv_empty[slot]);
+          ++p;
+          slot = p % C::NSLOT;
+          if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
+          tc_fence_after();
+          const uint32_t vaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
+          for (int s = 0; s < a.NT; ++s) {
+            if (!mbar_wait(&p_full[s], jt & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+            const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
+  #pragma unroll
+            for (int k = 0; k < BN / C::UK; ++k) {
+              // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with
+              // 4-row atoms (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
+              const uint64_t bd = DT == 0 ? smem_desc(vaddr + k * C::UK * 128, BN * 128, 512, 1u)
+                                          : smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
+              if constexpr (DT == 2) {
+                umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+                umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
+              } else {
+                umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+              }
+            }
+            umma_commit(&o_done[s]);
+          }
+          if (!ok) break;
+          umma_commit(&kv_empty[slot]);
           ++p;
         }
-        if (stop) break;
+        umma_commit(mma_done);
+        mbar_wait_drain(mma_done, 0, a.status);
       }
-      // Never leave with copies in flight.
-      for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status);
-      for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status);
     }
-  } else if (warp == 9) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = true;
-      for (int s = 0; s < a.NT && ok; ++s) ok = mbar_wait(&q_full[s], 0, abort_flag, a.status);
-      tc_fence_after();
-      int p = 0;
+  } else {
+    setmaxnreg_inc<C::REG_HIGH>();
+    if (warp < 4 * a.NT) {
+      // ---------------------------------------------------------------- softmax / epilogue
+      const int s = warp >> 2, qd = warp & 3;
+      const int rt = qd * 32 + lane;
+      constexpr int HS = 128 / BN;
+      const int hs = rt / BN, tl = rt % BN;
+      const int hl = (part * a.NT + s) * HS + hs;
+      const bool row_ok = (hl < a.G) && (i * BN + tl < L);
+      const int h = g * a.G + min(hl, a.G - 1);
+      const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+      const uint32_t s_addr = tmem + lane_base + (s ? C::S_COL1 : C::S_COL0);
+      const uint32_t o_addr = tmem + lane_base + (s ? C::O_COL1 : C::O_COL0);
+      const float s2 = a.sm_scale_log2;
+      const float bias_raw = a.log2_blk / s2;
+      float m_run = -CUDART_INF_F, l_run = 0.f;
+      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status));
+      int done_tiles = 0;
       for (int jt = 0; jt < n_tiles && ok; ++jt) {
-        int slot = p % C::NSLOT;
-        if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
-        tc_fence_after();
-        const uint32_t kaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
-        for (int s = 0; s < a.NT; ++s) {
-          if (jt > 0 && !mbar_wait(&o_done[s], (jt - 1) & 1, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t qaddr = sbase + C::OFF_Q + s * C::Q_BYTES;
-          const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
-#pragma unroll
-          for (int k = 0; k < D / C::UK; ++k) {
-            const int c = (k * C::UK) / C::KCH;
-            const int koff = ((k * C::UK) % C::KCH) * C::ELT;
-            const uint64_t ad = smem_desc_sw128(qaddr + c * (128 * 128) + koff, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(kaddr + c * (BN * 128) + koff, 16, 1024);
-            umma_ss<C::KIND>(dcol, ad, bd, C::IDESC_S, k > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[s]);
-        }
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jt & 1, abort_flag, a.status));
         if (!ok) break;
-        umma_commit(&kv_empty[slot]);
-        ++p;
-        slot = p % C::NSLOT;
-        if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
         tc_fence_after();
-        const uint32_t vaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
-        for (int s = 0; s < a.NT; ++s) {
-          if (!mbar_wait(&p_full[s], jt & 1, abort_flag, a.status)) {
-            ok = false;
-            break;
+        // The whole S row of this thread, in registers.
+        uint32_t v[BN];
+        if constexpr (BN == 128)
+          tmem_ld128_sync(s_addr, v);
+        else
+          tmem_ld64_sync(s_addr, v);
+        // Tile kinds: virtual (pooled keys of blocks [jt*BN, jt*BN+BN): only pruned blocks, with the
+        // ln n_j bias), diagonal (causal mask), full (no mask).  The mask works on raw S values:
+        // x = S * s2 with s2 > 0, so the bias is added as log2(n)/s2 and the max is taken on raw S.
+        float xs[BN];
+        if (jt < n_virt) {
+  #pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            const uint32_t word = pruned_word(kmask, jt * BN + c * 32, i);
+  #pragma unroll
+            for (int e = 0; e < 32; ++e)
+              xs[c * 32 + e] = ((word >> e) & 1u) ? __uint_as_float(v[c * 32 + e]) + bias_raw : -CUDART_INF_F;
           }
-          tc_fence_after();
-          const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
-          const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
-#pragma unroll
-          for (int k = 0; k < BN / C::UK; ++k) {
-            // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with
-            // 4-row atoms (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
-            const uint64_t bd = DT == 0 ? smem_desc(vaddr + k * C::UK * 128, BN * 128, 512, 1u)
-                                        : smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
-            if constexpr (DT == 2) {
-              umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-              umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
-            } else {
-              umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+        } else if (jt == n_tiles - 1) {
+  #pragma unroll
+          for (int e = 0; e < BN; ++e) xs[e] = (e <= tl) ? __uint_as_float(v[e]) : -CUDART_INF_F;
+        } else {
+  #pragma unroll
+          for (int e = 0; e < BN; ++e) xs[e] = __uint_as_float(v[e]);
+        }
+        float m4[4] = {xs[0], xs[1], xs[2], xs[3]};
+  #pragma unroll
+        for (int e = 4; e < BN; e += 4) {
+          m4[0] = fmaxf(m4[0], xs[e]);
+          m4[1] = fmaxf(m4[1], xs[e + 1]);
+          m4[2] = fmaxf(m4[2], xs[e + 2]);
+          m4[3] = fmaxf(m4[3], xs[e + 3]);
+        }
+        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * s2;
+        const float m_new = fmaxf(m_run, mt);
+        const bool need = m_new > m_run + C::LAZY;
+        if (jt > 0 && __any_sync(0xFFFFFFFFu, need)) {
+          const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32_sync(o_addr + c * 32, o);
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(o_addr + c * 32, o);
+          }
+          tmem_st_wait();
+        }
+        if (need) {
+          l_run = (m_run == -CUDART_INF_F) ? 0.f : l_run * fast_exp2(m_run - m_new);
+          m_run = m_new;
+        }
+        // P = 2^(S*s2 - m + P_SHIFT), packed to the MMA operand type and written over S in TMEM.
+        const float nmu = C::P_SHIFT - ((m_run == -CUDART_INF_F) ? 0.f : m_run);
+        float rs[2] = {0.f, 0.f};
+        if constexpr (DT == 1) {
+          uint32_t pk[BN / 2];
+  #pragma unroll
+          for (int e = 0; e < BN / 2; ++e) {
+            const float p0 = fast_exp2(fmaf(xs[2 * e], s2, nmu));
+            const float p1 = fast_exp2(fmaf(xs[2 * e + 1], s2, nmu));
+            rs[0] += p0;
+            rs[1] += p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+  #pragma unroll
+          for (int c = 0; c < BN / 64; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
+        } else if constexpr (DT == 2) {
+          // K-step c (32 keys) of the PV MMA: hi plane at columns [16c, 16c+8), lo at [16c+8, 16c+16).
+          uint32_t pk[BN / 2];
+  #pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float q4[4];
+  #pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                q4[u] = fast_exp2(fmaf(xs[c * 32 + 4 * e + u], s2, nmu));
+                rs[u & 1] += q4[u];
+              }
+              split_e4m3x4(q4[0], q4[1], q4[2], q4[3], pk[c * 16 + e], pk[c * 16 + 8 + e]);
             }
           }
-          umma_commit(&o_done[s]);
+  #pragma unroll
+          for (int c = 0; c < BN / 64; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
+        } else {
+          uint32_t pk[BN];
+  #pragma unroll
+          for (int e = 0; e < BN; ++e) {
+            const float p0 = fast_exp2(fmaf(xs[e], s2, nmu));
+            rs[e & 1] += p0;
+            pk[e] = __float_as_uint(p0);
+          }
+  #pragma unroll
+          for (int c = 0; c < BN / 32; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
         }
-        if (!ok) break;
-        umma_commit(&kv_empty[slot]);
-        ++p;
+        const float rsum = rs[0] + rs[1];
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[s]);
+        l_run += rsum;
+        done_tiles = jt + 1;
       }
-      umma_commit(mma_done);
-      mbar_wait_drain(mma_done, 0, a.status);
-    }
-  } else if (warp < 4 * a.NT) {
-    // ---------------------------------------------------------------- softmax / epilogue
-    const int s = warp >> 2, qd = warp & 3;
-    const int rt = qd * 32 + lane;
-    constexpr int HS = 128 / BN;
-    const int hs = rt / BN, tl = rt % BN;
-    const int hl = (part * a.NT + s) * HS + hs;
-    const bool row_ok = (hl < a.G) && (i * BN + tl < L);
-    const int h = g * a.G + min(hl, a.G - 1);
-    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-    const uint32_t s_addr = tmem + lane_base + (s ? C::S_COL1 : C::S_COL0);
-    const uint32_t o_addr = tmem + lane_base + (s ? C::O_COL1 : C::O_COL0);
-    float m_run = -CUDART_INF_F, l_run = 0.f;
-    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status));
-    int done_tiles = 0;
-    for (int jt = 0; jt < n_tiles && ok; ++jt) {
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jt & 1, abort_flag, a.status));
-      if (!ok) break;
+      if (ok && done_tiles == n_tiles)
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_tiles - 1) & 1, abort_flag, a.status));
       tc_fence_after();
-      // Kind of tile: virtual (pooled keys of blocks [jt*BN, jt*BN+BN)), diagonal, or full.
-      const bool virt = jt < n_virt;
-      const bool diag = !virt && jt == n_tiles - 1;
-      // Pass 1: masked row max of this tile, 32 columns at a time straight from TMEM.
-      float mt = -CUDART_INF_F;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(s_addr + c * 32, v);
-        const uint32_t mword = virt ? pruned_word(kmask, jt * BN + c * 32, i) : 0u;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float xv = logit(v[e], a.sm_scale_log2, virt, diag, mword, e, c * 32 + e, tl, a.log2_blk);
-          mt = fmaxf(mt, xv);
-        }
-      }
-      const float m_new = fmaxf(m_run, mt);
-      const bool need = m_new > m_run + C::LAZY;
-      if (jt > 0 && __any_sync(0xFFFFFFFFu, need)) {
-        const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
-#pragma unroll
+      if (ok) {
+        const int tok = P.tok_off[r] + i * BN + tl;
+        const float inv = a.v_descale / l_run;
+  #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
           tmem_ld32_sync(o_addr + c * 32, v);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-          tmem_st32(o_addr + c * 32, v);
-        }
-        tmem_st_wait();
-      }
-      if (need) {
-        l_run = (m_run == -CUDART_INF_F) ? 0.f : l_run * fast_exp2(m_run - m_new);
-        m_run = m_new;
-      }
-      const float mu = ((m_run == -CUDART_INF_F) ? 0.f : m_run) - C::P_SHIFT;
-      // Pass 2: P = 2^(x - m), packed to the MMA type and written over the columns of S
-      // already consumed (chunk c of P lands at or before chunk c of S).
-      float rsum = 0.f;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(s_addr + c * 32, v);
-        const uint32_t mword = virt ? pruned_word(kmask, jt * BN + c * 32, i) : 0u;
-        float pv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          pv[e] = fast_exp2(logit(v[e], a.sm_scale_log2, virt, diag, mword, e, c * 32 + e, tl, a.log2_blk) - mu);
-          rsum += pv[e];
-        }
-        if constexpr (DT == 1) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
-          tmem_st16(s_addr + c * 16, pk);
-        } else if constexpr (DT == 2) {
-          // K-step c of the PV MMA: hi plane at columns [16c, 16c+8), lo plane at [16c+8, 16c+16).
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            split_e4m3x4(pv[4 * e], pv[4 * e + 1], pv[4 * e + 2], pv[4 * e + 3], pk[e], pk[8 + e]);
-          tmem_st16(s_addr + c * 16, pk);
-        } else {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = __float_as_uint(pv[e]);
-          tmem_st32(s_addr + c * 32, pk);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[s]);
-      l_run += rsum;
-      done_tiles = jt + 1;
-    }
-    if (ok && done_tiles == n_tiles)
-      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_tiles - 1) & 1, abort_flag, a.status));
-    tc_fence_after();
-    if (ok) {
-      const int tok = P.tok_off[r] + i * BN + tl;
-      const float inv = a.v_descale / l_run;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32_sync(o_addr + c * 32, v);
-        if (row_ok) {
-          if constexpr (DT == 0) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+          if (row_ok) {
+            if constexpr (DT == 0) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                                      (static_cast<int64_t>(tok) * a.Hq + h) * D + c * 32);
+  #pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                     __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
                                                     (static_cast<int64_t>(tok) * a.Hq + h) * D + c * 32);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
-                                   __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
-                                                  (static_cast<int64_t>(tok) * a.Hq + h) * D + c * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv, __uint_as_float(v[8 * e + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv);
-              dst[e] = w;
+  #pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(v[8 * e + 0]) * inv, __uint_as_float(v[8 * e + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(v[8 * e + 2]) * inv, __uint_as_float(v[8 * e + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(v[8 * e + 4]) * inv, __uint_as_float(v[8 * e + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(v[8 * e + 6]) * inv, __uint_as_float(v[8 * e + 7]) * inv);
+                dst[e] = w;
+              }
             }
           }
         }
+        if (row_ok && a.lse != nullptr)
+          a.lse[static_cast<int64_t>(h) * a.total_tokens + tok] =
+              (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f;
       }
-      if (row_ok && a.lse != nullptr)
-        a.lse[static_cast<int64_t>(h) * a.total_tokens + tok] =
-            (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f;
     }
   }
 
@@ -470,7 +539,7 @@ static cudaError_t launch_one(const AttnArgs& a, const Fp2Plan& P, int64_t items
   cudaError_t e = cudaFuncSetAttribute(attention_kernel<DT, D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  attention_kernel<DT, D, BN><<<static_cast<unsigned>(items), 320, C::SMEM_BYTES, stream>>>(a, P);
+  attention_kernel<DT, D, BN><<<static_cast<unsigned>(items), 384, C::SMEM_BYTES, stream>>>(a, P);
   return cudaGetLastError();
 }
 
