@@ -295,67 +295,90 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else if (warp == 9) {
       // ---------------------------------------------------------------- MMA issuer
+      // Ping-pong order per key tile j: QK0(j), PV1(j-1), QK1(j), PV0(j).  The softmax of tile 0
+      // then runs while the tensor pipe does PV1(j-1) and QK1(j), and the softmax of tile 1 while
+      // it does PV0(j) and QK0(j+1), so the two softmax warpgroups alternate instead of competing.
       if (lane == 0) {
         bool ok = true;
         for (int s = 0; s < a.NT && ok; ++s) ok = mbar_wait(&q_full[s], 0, abort_flag, a.status);
         tc_fence_after();
+        // Descriptors are formed once per tile; a K step only moves the start address, which is
+        // the low 14 bits (address >> 4) of the descriptor and cannot carry (shared memory < 256 KB).
+        auto issue_qk = [&](int s, uint32_t kaddr) {
+          const uint64_t ad0 = smem_desc_sw128(sbase + C::OFF_Q + s * C::Q_BYTES, 16, 1024);
+          const uint64_t bd0 = smem_desc_sw128(kaddr, 16, 1024);
+          const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+#pragma unroll 1
+          for (int k = 0; k < D / C::UK; ++k) {
+            const int c = (k * C::UK) / C::KCH;
+            const int koff = ((k * C::UK) % C::KCH) * C::ELT;
+            umma_ss<C::KIND>(dcol, ad0 + static_cast<uint64_t>((c * (128 * 128) + koff) >> 4),
+                             bd0 + static_cast<uint64_t>((c * (BN * 128) + koff) >> 4), C::IDESC_S, k > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[s]);
+        };
+        auto issue_pv = [&](int s, uint32_t vaddr, int jt) {
+          const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+          const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
+          // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with 4-row atoms
+          // (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
+          const uint64_t vd0 = DT == 0 ? smem_desc(vaddr, BN * 128, 512, 1u) : smem_desc_sw128(vaddr, BN * 128, 1024);
+#pragma unroll 1
+          for (int k = 0; k < BN / C::UK; ++k) {
+            const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::UK * 128) >> 4);
+            if constexpr (DT == 2) {
+              umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+              umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
+            } else {
+              umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+            }
+          }
+          umma_commit(&o_done[s]);
+        };
         int p = 0;
+        int vslot_prev = 0;
+        uint32_t vaddr_prev = 0;
         for (int jt = 0; jt < n_tiles && ok; ++jt) {
-          int slot = p % C::NSLOT;
-          if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
-          tc_fence_after();
-          const uint32_t kaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
-          for (int s = 0; s < a.NT; ++s) {
-            if (jt > 0 && !mbar_wait(&o_done[s], (jt - 1) & 1, abort_flag, a.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t qaddr = sbase + C::OFF_Q + s * C::Q_BYTES;
-            const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
-  #pragma unroll
-            for (int k = 0; k < D / C::UK; ++k) {
-              const int c = (k * C::UK) / C::KCH;
-              const int koff = ((k * C::UK) % C::KCH) * C::ELT;
-              const uint64_t ad = smem_desc_sw128(qaddr + c * (128 * 128) + koff, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(kaddr + c * (BN * 128) + koff, 16, 1024);
-              umma_ss<C::KIND>(dcol, ad, bd, C::IDESC_S, k > 0 ? 1u : 0u);
-            }
-            umma_commit(&s_full[s]);
-          }
-          if (!ok) break;
-          umma_commit(&kv_empty[slot]);
+          const int kslot = p % C::NSLOT;
+          if (!mbar_wait(&kv_full[kslot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
           ++p;
-          slot = p % C::NSLOT;
-          if (!mbar_wait(&kv_full[slot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
           tc_fence_after();
-          const uint32_t vaddr = sbase + C::OFF_KV + slot * C::KV_BYTES;
-          for (int s = 0; s < a.NT; ++s) {
-            if (!mbar_wait(&p_full[s], jt & 1, abort_flag, a.status)) {
-              ok = false;
-              break;
+          const uint32_t kaddr = sbase + C::OFF_KV + kslot * C::KV_BYTES;
+          if (jt > 0 && !mbar_wait(&o_done[0], (jt - 1) & 1, abort_flag, a.status)) break;
+          tc_fence_after();
+          issue_qk(0, kaddr);
+          if (a.NT == 2) {
+            if (jt > 0) {
+              if (!mbar_wait(&p_full[1], (jt - 1) & 1, abort_flag, a.status)) break;
+              tc_fence_after();
+              issue_pv(1, vaddr_prev, jt - 1);
+              umma_commit(&kv_empty[vslot_prev]);
+              if (!mbar_wait(&o_done[1], (jt - 1) & 1, abort_flag, a.status)) break;
+              tc_fence_after();
             }
-            tc_fence_after();
-            const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
-            const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
-  #pragma unroll
-            for (int k = 0; k < BN / C::UK; ++k) {
-              // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with
-              // 4-row atoms (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
-              const uint64_t bd = DT == 0 ? smem_desc(vaddr + k * C::UK * 128, BN * 128, 512, 1u)
-                                          : smem_desc_sw128(vaddr + k * C::UK * 128, BN * 128, 1024);
-              if constexpr (DT == 2) {
-                umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-                umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
-              } else {
-                umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-              }
-            }
-            umma_commit(&o_done[s]);
+            issue_qk(1, kaddr);
           }
-          if (!ok) break;
-          umma_commit(&kv_empty[slot]);
+          umma_commit(&kv_empty[kslot]);
+          const int vslot = p % C::NSLOT;
+          if (!mbar_wait(&kv_full[vslot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
           ++p;
+          tc_fence_after();
+          const uint32_t vaddr = sbase + C::OFF_KV + vslot * C::KV_BYTES;
+          if (!mbar_wait(&p_full[0], jt & 1, abort_flag, a.status)) break;
+          tc_fence_after();
+          issue_pv(0, vaddr, jt);
+          if (a.NT == 2) {
+            vslot_prev = vslot;
+            vaddr_prev = vaddr;
+          } else {
+            umma_commit(&kv_empty[vslot]);
+          }
+          if (jt == n_tiles - 1 && a.NT == 2) {
+            if (!mbar_wait(&p_full[1], jt & 1, abort_flag, a.status)) break;
+            tc_fence_after();
+            issue_pv(1, vaddr, jt);
+            umma_commit(&kv_empty[vslot]);
+          }
         }
         umma_commit(mma_done);
         mbar_wait_drain(mma_done, 0, a.status);
