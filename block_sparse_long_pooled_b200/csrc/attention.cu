@@ -344,8 +344,10 @@ __global__ void __launch_bounds__(384, 1)
           ++p;
           tc_fence_after();
           const uint32_t kaddr = sbase + C::OFF_KV + kslot * C::KV_BYTES;
-          if (jt > 0 && !mbar_wait(&o_done[0], (jt - 1) & 1, abort_flag, a.status)) break;
-          tc_fence_after();
+          // QK_s(j) is issued right behind PV_s(j-1) without waiting for it: the tensor pipe runs
+          // one thread's MMAs in issue order, so PV_s(j-1) has read P_s out of the S_s columns
+          // before QK_s(j) overwrites them, and s_full (a commit) also covers PV_s(j-1), so the
+          // softmax never sees O_s mid-update.
           issue_qk(0, kaddr);
           if (a.NT == 2) {
             if (jt > 0) {
@@ -353,8 +355,6 @@ __global__ void __launch_bounds__(384, 1)
               tc_fence_after();
               issue_pv(1, vaddr_prev, jt - 1);
               umma_commit(&kv_empty[vslot_prev]);
-              if (!mbar_wait(&o_done[1], (jt - 1) & 1, abort_flag, a.status)) break;
-              tc_fence_after();
             }
             issue_qk(1, kaddr);
           }
