@@ -346,6 +346,66 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ sweeps (ablations)
+
+def run_sweep(kind, args):
+    """Sweeps on the 64K FP8 workload (one JSON line per point).
+
+    alpha:       block density and step / attention time for alpha in {0.2, 0.1, 0.05, 0.025, 0.0125}
+                 (the paper page's Table 9 grid).
+    correction:  attention time with mean correction on and off, and the relative L2 error of
+                 each against the all-blocks-kept output of the same library (Figure 6, Table 8).
+    sparsity:    attention time against density over a wide alpha range, next to the time the
+                 computed tiles would take at the measured tensor peak (Figure 5).
+    """
+    import torch
+    from block_sparse_long_pooled_b200 import build, fp2
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    wname = args.workload if args.workload != DEFAULT_WORKLOAD else "qwen4b_64k_e4m3"
+    peak = peaks["bf16_tflops_sustained"] * (2.0 if "e4m3" in wname else 1.0)
+    base = Path(wname, dev)
+    steps, warm = max(5, args.steps // 2), max(3, args.warmup)
+
+    def measure(path):
+        ms, st = time_path(path, steps, warm)
+        ach, kept, pruned, causal = path.achieved_flops()
+        return {"ms_per_step": ms / steps, "attend_ms": st["attend"], "density": kept / causal,
+                "attend_tflops": ach / (st["attend"] * 1e-3) / 1e12,
+                "ideal_attend_ms": ach / (peak * 1e12) * 1e3}
+
+    def retarget(alpha=None, correction=None):
+        w = base.w
+        base.params = fp2.make_params(w.block_size, w.alpha if alpha is None else alpha, w.sink_blocks,
+                                      w.window_blocks, w.last_n_blocks, w.min_sparse_len,
+                                      w.mean_correction if correction is None else correction)
+        base.w = w.replace(alpha=base.w.alpha if alpha is None else alpha,
+                           mean_correction=w.mean_correction if correction is None else correction)
+
+    out = []
+    if kind in ("alpha", "sparsity"):
+        grid = [0.2, 0.1, 0.05, 0.025, 0.0125] if kind == "alpha" else \
+            [0.9, 0.5, 0.2, 0.1, 0.05, 0.02, 0.01, 0.005, 0.002, 0.001, 1e-4, 0.0]
+        for al in grid:
+            retarget(alpha=al)
+            out.append({"sweep": kind, "workload": wname, "alpha": al, **measure(base)})
+    elif kind == "correction":
+        retarget(alpha=0.0)
+        base.step()
+        dense = base.out.float().clone()
+        for corr in (True, False):
+            retarget(alpha=0.1, correction=corr)
+            m = measure(base)
+            o = base.out.float()
+            m["rel_l2_vs_all_kept"] = float(torch.linalg.vector_norm(o - dense) / torch.linalg.vector_norm(dense))
+            m["max_abs_vs_all_kept"] = float((o - dense).abs().max())
+            out.append({"sweep": kind, "workload": wname, "alpha": 0.1, "mean_correction": corr, **m})
+    for line in out:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -356,7 +416,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-extras", action="store_true", help="skip the FP8, all-kept, e2e and CPU legs")
+    ap.add_argument("--sweep", choices=["alpha", "correction", "sparsity"], default=None,
+                    help="ablation sweeps on the 64K FP8 workload instead of the benchmark line")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args.sweep, args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

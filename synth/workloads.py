@@ -108,6 +108,11 @@ WORKLOADS = {
     "qwen30b_64k_paged_bf16": _w("qwen30b_64k_paged_bf16", seqlens=(65536,), num_q_heads=32, num_kv_heads=4,
                                  head_dim=128, block_size=128, dtype="bf16", paged=True, page_size=64, seed=4,
                                  description="Qwen3-30B-A3B-shaped layer, seq 65536, GQA 8, paged KV (64-token pages)"),
+    # Qwen3-4B-shaped layer at 64K in FP8: the setting of the paper page's Table 9 (alpha sweep) and
+    # Figures 5-6 (latency vs sparsity, correction overhead); used by the sweeps, not a parity config.
+    "qwen4b_64k_e4m3": _w("qwen4b_64k_e4m3", seqlens=(65536,), num_q_heads=32, num_kv_heads=8, head_dim=128,
+                          block_size=128, dtype="e4m3", seed=6,
+                          description="Qwen3-4B-shaped layer, seq 65536, GQA 4, d 128, block 128, FP8 e4m3"),
     "varlen6_paged_e4m3": _w("varlen6_paged_e4m3", seqlens=(2048, 4096, 16384, 32768, 65536, 131072),
                              num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=128, dtype="e4m3",
                              paged=True, page_size=64, min_sparse_len=8192, seed=5,
