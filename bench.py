@@ -34,10 +34,10 @@ UNIT = "TFLOP/s (dense-equivalent)"
 DEFAULT_WORKLOAD = "llama8b_128k_bf16"
 FP8_WORKLOAD = "llama8b_128k_e4m3"
 
-# DRAM traffic of one attention launch on the 128K bf16 workload, from an ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the kernel source it was
-# taken on (sha256 prefix of csrc/attention.cu).  None until captured.
-ATTN_TRAFFIC = {"bytes": None, "source_sha": None}
+# DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
+# taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7335059200 + 1036489728, "source_sha": "b7f4311132b81344"}}
 
 
 def source_sha(path):
@@ -468,7 +468,8 @@ def main():
     peak_bf16 = peaks["bf16_tflops_sustained"]
     peak = peak_bf16 if w.dtype != "e4m3" else 2.0 * peak_bf16
     sha = source_sha(os.path.join(ROOT, "block_sparse_long_pooled_b200", "csrc", "attention.cu"))
-    traffic = ATTN_TRAFFIC["bytes"] if ATTN_TRAFFIC["source_sha"] == sha else None
+    tr = ATTN_TRAFFIC.get(w.name)
+    traffic = tr["bytes"] if tr is not None and tr["source_sha"] == sha else None
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
