@@ -35,8 +35,14 @@ Readings of the pages that this oracle fixes (the CUDA path takes the same):
   min_sparse_len; j < sink; j > i - max(window, 1) (the diagonal block is
   always exact); every j of the last ``last_n`` query blocks.
 * Mean correction uses the token's own query: a pruned block j contributes the
-  logit q_t . kbar_j * scale + ln n_j with value vbar_j.  With q_len == kv_len
-  every pruned block lies strictly left of the window, so it is fully visible.
+  logit q_t . kbar_j * scale + ln n_j with value vbar_j.  Every pruned block lies
+  strictly left of the diagonal, so it is fully visible.
+* Chunked prefill (the paper page's Table 6; ResearchPod: discovery re-runs per
+  chunk): a query chunk is the last L_q tokens of a sequence whose keys number
+  L_k >= L_q, with bottom-right causal alignment (chunk token t sits at absolute
+  position L_k - L_q + t).  The chunk must start on a block boundary, so chunk
+  block i is absolute block I = (L_k - L_q)/B + i; causality, the diagonal and the
+  window refer to I; last_n and min_sparse_len refer to the chunk's queries.
 
 Parity pins: tests/test_oracle_pins.py checks these functions against dense
 softmax attention from torch (alpha = 0), the closed form in which mean
@@ -122,52 +128,65 @@ def gather_paged(cache: np.ndarray, page_table: np.ndarray, seqlens: Sequence[in
     return np.concatenate(parts)
 
 
-def block_scores(qbar: np.ndarray, kbar: np.ndarray, scale: float) -> np.ndarray:
-    """Pooled block scores of one sequence: s[h, i, j] = qbar[i,h] . kbar[j,g(h)] * scale, j <= i.
+def _causal(Nq: int, Nk: int, off: int) -> np.ndarray:
+    """[Nq, Nk] boolean: key block j is visible from query block i (absolute block i + off)."""
+    return np.arange(Nk)[None, :] <= (np.arange(Nq)[:, None] + off)
 
-    qbar: [N, Hq, d]; kbar: [N, Hkv, d].  Entries with j > i are -inf.
+
+def block_scores(qbar: np.ndarray, kbar: np.ndarray, scale: float, q_block_offset: int = 0) -> np.ndarray:
+    """Pooled block scores of one sequence: s[h, i, j] = qbar[i,h] . kbar[j,g(h)] * scale, j <= i + off.
+
+    qbar: [Nq, Hq, d]; kbar: [Nk, Hkv, d]; q_block_offset = prefix blocks before the query chunk
+    (0 for a whole-sequence prefill, where Nq = Nk).  Entries with j > i + off are -inf.
     """
-    N, Hq, _ = qbar.shape
-    Hkv = kbar.shape[1]
+    Nq, Hq, _ = qbar.shape
+    Nk, Hkv = kbar.shape[0], kbar.shape[1]
     G = Hq // Hkv
-    s = np.empty((Hq, N, N), dtype=np.float64)
+    s = np.empty((Hq, Nq, Nk), dtype=np.float64)
     for h in range(Hq):
         s[h] = (qbar[:, h, :] @ kbar[:, h // G, :].T) * scale
-    s[:, ~np.tri(N, dtype=bool)] = -np.inf
+    s[:, ~_causal(Nq, Nk, q_block_offset)] = -np.inf
     return s
 
 
-def forced_blocks(N: int, L: int, p: SparseParams) -> np.ndarray:
-    """Blocks kept regardless of score, as a causal [N, N] boolean (i = query block, j = key block)."""
+def forced_blocks(N: int, L: int, p: SparseParams, Nk: Optional[int] = None, q_block_offset: int = 0) -> np.ndarray:
+    """Blocks kept regardless of score, as a causal [N, Nk] boolean (i = query block, j = key block).
+
+    N, L: query blocks and query tokens of the sequence (or chunk); the query block i sits at
+    absolute block i + q_block_offset, which is what the window and the causal limit refer to;
+    last_n and min_sparse_len refer to the queries.
+    """
+    Nk = N if Nk is None else Nk
     i = np.arange(N)[:, None]
-    j = np.arange(N)[None, :]
-    causal = j <= i
+    I = i + q_block_offset
+    j = np.arange(Nk)[None, :]
+    causal = j <= I
     if L < p.min_sparse_len or p.alpha <= 0.0:
         return causal.copy()
-    f = (j < p.sink_blocks) | (j > i - max(p.window_blocks, 1)) | (i >= N - p.last_n_blocks)
+    f = (j < p.sink_blocks) | (j > I - max(p.window_blocks, 1)) | (i >= N - p.last_n_blocks)
     return f & causal
 
 
-def select_blocks(s: np.ndarray, num_kv_heads: int, L: int, p: SparseParams):
+def select_blocks(s: np.ndarray, num_kv_heads: int, L: int, p: SparseParams, q_block_offset: int = 0):
     """Max-based dynamic thresholding (abstract; Table 9) with the GQA union per KV head (Table 7).
 
-    s: [Hq, N, N] block scores of one sequence.  Returns (kept [Hkv, N, N],
-    borderline [Hkv, N, N]); a block is borderline when it is not forced and
-    some head of the group has |s - (rowmax + ln alpha)| < 1e-3.
+    s: [Hq, N, Nk] block scores of one sequence (or query chunk); L is its query token count.
+    Returns (kept [Hkv, N, Nk], borderline [Hkv, N, Nk]); a block is borderline when it is not
+    forced and some head of the group has |s - (rowmax + ln alpha)| < 1e-3.
     """
-    Hq, N, _ = s.shape
+    Hq, N, Nk = s.shape
     G = Hq // num_kv_heads
     if N == 0:
-        empty = np.zeros((num_kv_heads, 0, 0), dtype=bool)
+        empty = np.zeros((num_kv_heads, 0, Nk), dtype=bool)
         return empty, empty.copy()
-    forced = forced_blocks(N, L, p)
-    causal = np.tri(N, dtype=bool)
-    kept = np.zeros((num_kv_heads, N, N), dtype=bool)
-    border = np.zeros((num_kv_heads, N, N), dtype=bool)
+    forced = forced_blocks(N, L, p, Nk, q_block_offset)
+    causal = _causal(N, Nk, q_block_offset)
+    kept = np.zeros((num_kv_heads, N, Nk), dtype=bool)
+    border = np.zeros((num_kv_heads, N, Nk), dtype=bool)
     dense = L < p.min_sparse_len or p.alpha <= 0.0
     for g in range(num_kv_heads):
         keep_g = forced.copy()
-        bord_g = np.zeros((N, N), dtype=bool)
+        bord_g = np.zeros((N, Nk), dtype=bool)
         if not dense:
             for h in range(g * G, (g + 1) * G):
                 rowmax = s[h].max(axis=1)                       # over j <= i (others are -inf)
@@ -197,12 +216,13 @@ def csr_from_kept(kept_per_seq: Sequence[np.ndarray]):
     return row_ptr, col_idx
 
 
-def kept_from_csr(row_ptr, col_idx, seqlens, B, Hkv):
-    """Inverse of csr_from_kept: per-sequence kept [Hkv, N, N] booleans."""
+def kept_from_csr(row_ptr, col_idx, seqlens, B, Hkv, seqlens_k=None):
+    """Inverse of csr_from_kept: per-sequence kept [Hkv, Nq, Nk] booleans."""
     out, row = [], 0
-    for L in seqlens:
+    for r, L in enumerate(seqlens):
         N = num_blocks(L, B)
-        kept = np.zeros((Hkv, N, N), dtype=bool)
+        Nk = num_blocks(seqlens_k[r], B) if seqlens_k is not None else N
+        kept = np.zeros((Hkv, N, Nk), dtype=bool)
         for i in range(N):
             for g in range(Hkv):
                 kept[g, i, col_idx[row_ptr[row]:row_ptr[row + 1]]] = True
@@ -213,7 +233,7 @@ def kept_from_csr(row_ptr, col_idx, seqlens, B, Hkv):
 
 def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correction: bool,
            rows: Optional[np.ndarray] = None, head_ids: Optional[Sequence[int]] = None,
-           group: Optional[int] = None):
+           group: Optional[int] = None, q_offset: int = 0):
     """Exact attention over kept blocks plus mean correction for pruned ones, one sequence.
 
     Figure 4 caption: selected blocks are computed exactly; each pruned block J
@@ -226,18 +246,23 @@ def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correct
         O_t = (sum e^{z-m} v_u + sum e^{c-m} vbar_j) / (sum e^{z-m} + sum e^{c-m})
         LSE_t = m + ln(denominator)
 
-    q: [L, Hq, d]; k, v: [L, Hkv, d]; kbar, vbar: [N, Hkv, d]; counts: [N];
-    kept: [Hkv, N, N].  rows: optional int array [n, 2] of (t, h) pairs; when
+    q: [Lq, Hq, d] at absolute positions q_offset + t (q_offset = the chunk's prefix length, a
+    multiple of B; 0 for a whole sequence); k, v: [Lk, Hkv, d]; kbar, vbar: [Nk, Hkv, d];
+    counts: [Nk]; kept: [Hkv, Nq, Nk].  rows: optional int array [n, 2] of (t, h) pairs; when
     given only those outputs are computed and O is [n, d], LSE [n].
     Otherwise O is [L, Hq, d] and LSE [Hq, L].  head_ids / group: when q holds
     only some query heads, head_ids[x] is the global head of q[:, x] and group
     is G; rows then index q's own head axis.
     """
     L, Hq, d = q.shape
+    Lk = k.shape[0]
     Hkv = k.shape[1]
     G = group if group is not None else Hq // Hkv
     gid = (lambda x: int(head_ids[x]) // G) if head_ids is not None else (lambda x: x // G)
     N = num_blocks(L, B)
+    if q_offset % B != 0:
+        raise ValueError("the query chunk must start on a block boundary")
+    ob = q_offset // B
     logn = np.log(counts.astype(np.float64))
     if rows is None:
         O = np.zeros((L, Hq, d))
@@ -256,16 +281,17 @@ def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correct
                 work.append((int(h), int(i), rows[sel, 0], sel))
     for h, i, toks, dest in work:
         g = gid(h)
-        if not kept[g, i, i]:
+        I = i + ob                                                  # absolute query block
+        if not kept[g, i, I]:
             raise ValueError("the diagonal block must be kept (it is only partly visible)")
-        kj = np.nonzero(kept[g, i, : i + 1])[0]
-        key_idx = np.concatenate([np.arange(j * B, min(L, (j + 1) * B)) for j in kj])
+        kj = np.nonzero(kept[g, i, : I + 1])[0]
+        key_idx = np.concatenate([np.arange(j * B, min(Lk, (j + 1) * B)) for j in kj])
         qt = q[toks, h, :]                                          # [n, d]
         z = (qt @ k[key_idx, g, :].T) * scale                       # [n, nk]
-        z[key_idx[None, :] > toks[:, None]] = -np.inf               # causal
+        z[key_idx[None, :] > (toks[:, None] + q_offset)] = -np.inf  # causal, bottom-right aligned
         vals = v[key_idx, g, :]
         if mean_correction:
-            pj = np.array([j for j in range(i + 1) if not kept[g, i, j]], dtype=np.int64)
+            pj = np.array([j for j in range(I + 1) if not kept[g, i, j]], dtype=np.int64)
         else:
             pj = np.zeros(0, dtype=np.int64)
         if len(pj):
@@ -287,40 +313,49 @@ def attend(q, k, v, kbar, vbar, counts, kept, B: int, scale: float, mean_correct
 
 
 def prefill(q, k, v, cu_seqlens, num_kv_heads: int, p: SparseParams, k_cache=None, v_cache=None,
-            page_table=None, kept_override=None, attention: bool = True):
+            page_table=None, kept_override=None, attention: bool = True, cu_seqlens_k=None):
     """The whole path for a packed batch: pool -> score -> select -> CSR -> attend.
 
-    q: [T, Hq, d]; k, v: [T, Hkv, d] fp64 (ignored when a paged cache is given,
-    which is gathered through the page table first).  kept_override: optional
-    list of per-sequence kept arrays to attend on instead of the selected ones.
-    Returns a dict of every intermediate result.
+    q: [T, Hq, d]; k, v: [Tk, Hkv, d] fp64 (ignored when a paged cache is given,
+    which is gathered through the page table first).  cu_seqlens_k: key offsets when
+    queries are a chunk at the end of each sequence (chunked prefill: the query chunk of
+    sequence r is its last L_q tokens, and L_k - L_q must be a multiple of the block size);
+    None means q_len == kv_len.  kept_override: optional list of per-sequence kept arrays
+    to attend on instead of the selected ones.  Returns a dict of every intermediate result.
     """
     cu = [int(x) for x in cu_seqlens]
+    cuk = cu if cu_seqlens_k is None else [int(x) for x in cu_seqlens_k]
     seqlens = [cu[r + 1] - cu[r] for r in range(len(cu) - 1)]
+    seqlens_k = [cuk[r + 1] - cuk[r] for r in range(len(cuk) - 1)]
     if page_table is not None:
-        k = gather_paged(k_cache, page_table, seqlens)
-        v = gather_paged(v_cache, page_table, seqlens)
+        k = gather_paged(k_cache, page_table, seqlens_k)
+        v = gather_paged(v_cache, page_table, seqlens_k)
     d = q.shape[2]
     scale = p.softmax_scale if p.softmax_scale > 0 else 1.0 / math.sqrt(d)
     B = p.block_size
-    out = {"qbar": [], "kbar": [], "vbar": [], "counts": [], "scores": [], "kept": [], "borderline": []}
+    out = {"qbar": [], "kbar": [], "vbar": [], "counts": [], "scores": [], "kept": [], "borderline": [],
+           "q_offset": []}
     for r, L in enumerate(seqlens):
-        qs, ks, vs = q[cu[r]:cu[r + 1]], k[cu[r]:cu[r + 1]], v[cu[r]:cu[r + 1]]
-        qbar, counts = pool_blocks(qs, B)
-        kbar, _ = pool_blocks(ks, B)
+        off = seqlens_k[r] - L
+        if off < 0 or off % B != 0:
+            raise ValueError("each query chunk must end its sequence and start on a block boundary")
+        qs, ks, vs = q[cu[r]:cu[r + 1]], k[cuk[r]:cuk[r + 1]], v[cuk[r]:cuk[r + 1]]
+        qbar, _ = pool_blocks(qs, B)
+        kbar, counts = pool_blocks(ks, B)
         vbar, _ = pool_blocks(vs, B)
-        s = block_scores(qbar, kbar, scale)
-        kept, border = select_blocks(s, num_kv_heads, L, p)
+        s = block_scores(qbar, kbar, scale, off // B)
+        kept, border = select_blocks(s, num_kv_heads, L, p, off // B)
         for key, val in (("qbar", qbar), ("kbar", kbar), ("vbar", vbar), ("counts", counts),
-                         ("scores", s), ("kept", kept), ("borderline", border)):
+                         ("scores", s), ("kept", kept), ("borderline", border), ("q_offset", off)):
             out[key].append(val)
     out["row_ptr"], out["col_idx"] = csr_from_kept(out["kept"])
     if attention:
         Os, LSEs = [], []
         for r, L in enumerate(seqlens):
             kept = kept_override[r] if kept_override is not None else out["kept"][r]
-            O, LSE = attend(q[cu[r]:cu[r + 1]], k[cu[r]:cu[r + 1]], v[cu[r]:cu[r + 1]], out["kbar"][r],
-                            out["vbar"][r], out["counts"][r], kept, B, scale, p.mean_correction)
+            O, LSE = attend(q[cu[r]:cu[r + 1]], k[cuk[r]:cuk[r + 1]], v[cuk[r]:cuk[r + 1]], out["kbar"][r],
+                            out["vbar"][r], out["counts"][r], kept, B, scale, p.mean_correction,
+                            q_offset=out["q_offset"][r])
             Os.append(O)
             LSEs.append(LSE)
         out["O"] = np.concatenate(Os)

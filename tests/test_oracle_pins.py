@@ -384,3 +384,53 @@ def test_csr_layout_row_order():
     assert list(col_idx) == [0, 0, 0, 1, 1, 0, 0]
     back = O.kept_from_csr(row_ptr, col_idx, [2, 1], 1, 2)
     assert np.array_equal(back[0], kept0) and np.array_equal(back[1], kept1)
+
+
+# ---------------------------------------------------------------- chunked prefill (q_len < kv_len)
+
+def test_chunk_equals_last_rows_of_whole_sequence():
+    """Bottom-right alignment: a chunk's selection and output are the whole sequence's last rows."""
+    rng = np.random.default_rng(20)
+    L, B, Hq, Hkv, d = 100, 8, 4, 2, 6
+    q, k, v = rand_qkv(rng, L, Hq, Hkv, d)
+    q += np.repeat(rng.standard_normal((13, Hq, d)) * 2, B, axis=0)[:L]
+    k += np.repeat(rng.standard_normal((13, Hkv, d)) * 2, B, axis=0)[:L]
+    p = _params(block_size=B, alpha=0.3, sink_blocks=1, window_blocks=2, last_n_blocks=1)
+    whole = O.prefill(q, k, v, [0, L], Hkv, p)
+    for prefix in (0, 32, 64, 96):
+        ch = O.prefill(q[prefix:], k, v, [0, L - prefix], Hkv, p, cu_seqlens_k=[0, L])
+        assert np.array_equal(ch["kept"][0], whole["kept"][0][:, prefix // B:, :])
+        assert np.max(np.abs(ch["O"] - whole["O"][prefix:])) < 1e-13
+        assert np.max(np.abs(ch["LSE"] - whole["LSE"][:, prefix:])) < 1e-13
+    assert (~whole["kept"][0] & np.tri(13, dtype=bool)).any()
+
+
+def test_chunk_alpha_zero_equals_bottom_right_causal_attention():
+    rng = np.random.default_rng(21)
+    Lk, Lq, B, Hq, Hkv, d = 90, 26, 8, 4, 1, 5
+    q, _, _ = rand_qkv(rng, Lq, Hq, Hkv, d)
+    _, k, v = rand_qkv(rng, Lk, Hq, Hkv, d)
+    r = O.prefill(q, k, v, [0, Lq], Hkv, _params(block_size=B, alpha=0.0), cu_seqlens_k=[0, Lk])
+    allowed = np.arange(Lk)[None, :] <= (np.arange(Lq)[:, None] + (Lk - Lq))
+    ref = sdpa_dense(q, k, v, 1 / math.sqrt(d), np.broadcast_to(allowed, (Hq, Lq, Lk)).copy())
+    assert np.max(np.abs(r["O"] - ref)) < 1e-12
+
+
+def test_chunked_varlen_equals_per_sequence_and_rejects_misaligned_chunks():
+    rng = np.random.default_rng(22)
+    B, Hq, Hkv, d = 8, 2, 1, 4
+    lk, lq = [40, 75], [8, 19]
+    q, _, _ = rand_qkv(rng, sum(lq), Hq, Hkv, d)
+    _, k, v = rand_qkv(rng, sum(lk), Hq, Hkv, d)
+    cq, ck = np.concatenate([[0], np.cumsum(lq)]), np.concatenate([[0], np.cumsum(lk)])
+    p = _params(block_size=B, alpha=0.4)
+    both = O.prefill(q, k, v, cq, Hkv, p, cu_seqlens_k=ck)
+    for r in range(2):
+        one = O.prefill(q[cq[r]:cq[r + 1]], k[ck[r]:ck[r + 1]], v[ck[r]:ck[r + 1]], [0, lq[r]], Hkv, p,
+                        cu_seqlens_k=[0, lk[r]])
+        assert np.max(np.abs(one["O"] - both["O"][cq[r]:cq[r + 1]])) == 0.0
+    rp, ci = both["row_ptr"], both["col_idx"]
+    back = O.kept_from_csr(rp, ci, lq, B, Hkv, seqlens_k=lk)
+    assert all(np.array_equal(a, b) for a, b in zip(back, both["kept"]))
+    with pytest.raises(ValueError):
+        O.prefill(q[:5], k[:40], v[:40], [0, 5], Hkv, p, cu_seqlens_k=[0, 40])   # prefix 35 not a block multiple
