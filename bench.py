@@ -185,7 +185,7 @@ class Path:
         w = self.w
         elt = {"f32": 4, "bf16": 2, "e4m3": 1}[w.dtype]
         T = w.total_tokens
-        nb = self.ws.total_blocks
+        nb = self.ws.total_q_blocks  # q_len == kv_len in the benchmark workloads
         read = T * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * elt
         write = nb * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * 4 + 2 * nb * w.num_kv_heads * w.head_dim * elt
         return read + write
@@ -357,6 +357,7 @@ def run_sweep(kind, args):
                  each against the all-blocks-kept output of the same library (Figure 6, Table 8).
     sparsity:    attention time against density over a wide alpha range, next to the time the
                  computed tiles would take at the measured tensor peak (Figure 5).
+    chunked:     the 128K bf16 layer as 8K / 16K chunks versus one pass (Table 6).
     """
     import torch
     from block_sparse_long_pooled_b200 import build, fp2
@@ -366,6 +367,10 @@ def run_sweep(kind, args):
     peaks = load_peaks()
     wname = args.workload if args.workload != DEFAULT_WORKLOAD else "qwen4b_64k_e4m3"
     peak = peaks["bf16_tflops_sustained"] * (2.0 if "e4m3" in wname else 1.0)
+    if kind == "chunked":
+        for line in chunked_sweep(args, dev, peaks):
+            print(json.dumps(line), flush=True)
+        return
     base = Path(wname, dev)
     steps, warm = max(5, args.steps // 2), max(3, args.warmup)
 
@@ -406,6 +411,75 @@ def run_sweep(kind, args):
         print(json.dumps(line), flush=True)
 
 
+def chunked_sweep(args, dev, peaks):
+    """Chunked prefill of the 128K bf16 layer: the sequence is processed in chunks of 8K / 16K
+    tokens (each chunk's queries against all keys so far, bottom-right causal; pooled prefix K/V
+    reused from earlier chunks) and as one 128K pass.  Reports per chunk size the summed
+    pool / discover / attend time over all chunks and the share spent outside attention."""
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    from synth import workloads as W
+    w = W.WORKLOADS["llama8b_128k_bf16"]
+    inp = W.generate(w)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    L, B = w.seqlens[0], w.block_size
+    params = fp2.make_params(B, w.alpha, w.sink_blocks, w.window_blocks, w.last_n_blocks, w.min_sparse_len,
+                             w.mean_correction)
+    full = fp2.make_problem(q, k, v, [0, L], w.num_kv_heads)
+    ws_full = fp2.fp2_workspace_query(full, params)
+    _, pooled = fp2.alloc_pooled(ws_full, full, dev)
+    pst = fp2.fp2_pooled(*(pooled[n].data_ptr() for n in ("qbar", "kbar", "vbar", "kbar_mma", "vbar_mma")))
+    scratch = fp2.alloc_scratch(ws_full.prefill_scratch_bytes, dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lines = []
+    for C in (8192, 16384, L):
+        chunks = []
+        for s0 in range(0, L, C):
+            prob = fp2.make_problem(q[s0:s0 + C], k, v, [0, C], w.num_kv_heads, cu_seqlens_k=[0, s0 + C],
+                                    kv_prefix_pooled=s0 > 0)
+            ws = fp2.fp2_workspace_query(prob, params)
+            ist, ix = fp2.alloc_index(ws, dev)
+            chunks.append((prob, ist, ix, s0))
+
+        def run(evs=None):
+            for n, (prob, ist, _, s0) in enumerate(chunks):
+                if evs:
+                    evs[n][0].record()
+                fp2.fp2_pool(prob, params, pst, scratch)
+                if evs:
+                    evs[n][1].record()
+                fp2.fp2_discover(prob, params, pst, ist, scratch)
+                if evs:
+                    evs[n][2].record()
+                fp2.fp2_attend(prob, params, pst, ist, out[s0:s0 + C], None, scratch)
+                if evs:
+                    evs[n][3].record()
+
+        run()
+        torch.cuda.synchronize()
+        t_h = time.perf_counter()
+        run()
+        host_ms = (time.perf_counter() - t_h) * 1e3   # enqueue time of all chunks' calls
+        torch.cuda.synchronize()
+        reps = 3
+        tot = {"pool": 0.0, "discover": 0.0, "attend": 0.0}
+        per_chunk = [0.0] * len(chunks)
+        for _ in range(reps):
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in chunks]
+            run(evs)
+            torch.cuda.synchronize()
+            for n, e in enumerate(evs):
+                tot["pool"] += e[0].elapsed_time(e[1]) / reps
+                tot["discover"] += e[1].elapsed_time(e[2]) / reps
+                tot["attend"] += e[2].elapsed_time(e[3]) / reps
+                per_chunk[n] += e[2].elapsed_time(e[3]) / reps
+        total = sum(tot.values())
+        lines.append({"sweep": "chunked", "workload": w.name, "chunk": C, "chunks": len(chunks),
+                      "total_ms": total, "stages_ms": tot, "outside_attention_share": (total - tot["attend"]) / total,
+                      "host_enqueue_ms": host_ms, "attend_ms_per_chunk": [round(x, 4) for x in per_chunk]})
+    return lines
+
+
 # ------------------------------------------------------------------ main
 
 def main():
@@ -416,7 +490,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-extras", action="store_true", help="skip the FP8, all-kept, e2e and CPU legs")
-    ap.add_argument("--sweep", choices=["alpha", "correction", "sparsity"], default=None,
+    ap.add_argument("--sweep", choices=["alpha", "correction", "sparsity", "chunked"], default=None,
                     help="ablation sweeps on the 64K FP8 workload instead of the benchmark line")
     args = ap.parse_args()
     if args.sweep:

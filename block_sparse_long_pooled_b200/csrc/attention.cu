@@ -167,16 +167,18 @@ __global__ void __launch_bounds__(384, 1)
   int r, i, sub;
   if (!map_heavy_first(P, 1, a.Hkv * a.parts, blockIdx.x, r, i, sub)) return;
   const int g = sub / a.parts, part = sub % a.parts;
-  const int L = P.len[r];
+  const int L = P.len[r];                 // query tokens of the sequence (or chunk)
+  const int I = P.pre_blk[r] + i;         // absolute key block of query block i (the diagonal)
+  const int Lk = P.pre_blk[r] * BN + L;   // key tokens of the sequence
   const int64_t row = static_cast<int64_t>(P.blk_off[r] + i) * a.Hkv + g;
   const int rs = a.row_ptr[row], re = a.row_ptr[row + 1];
   const int nkept = re - rs;
-  if (nkept <= 0 || nkept > i + 1) {
+  if (nkept <= 0 || nkept > I + 1) {
     if (tid == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
     return;
   }
-  const int npruned = i + 1 - nkept;
-  const int n_virt = (a.mean_correction && npruned > 0) ? (i + BN - 1) / BN : 0;
+  const int npruned = I + 1 - nkept;
+  const int n_virt = (a.mean_correction && npruned > 0) ? (I + BN - 1) / BN : 0;
   const int n_tiles = n_virt + nkept;
 
   if (warp == 0) {
@@ -214,19 +216,19 @@ __global__ void __launch_bounds__(384, 1)
     setmaxnreg_dec<C::REG_LOW>();
     if (warp == 8) {
       // ---------------------------------------------------------------- producer
-      const int nw = (i + 32) / 32;
+      const int nw = (I + 32) / 32;
       for (int w = lane; w < nw; w += 32) kmask[w] = 0u;
       __syncwarp();
       bool bad = false;
       for (int e = lane; e < nkept; e += 32) {
         const int j = a.col_idx[rs + e];
         const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
-        if (j < 0 || j > i || j <= prev)
+        if (j < 0 || j > I || j <= prev)
           bad = true;
         else
           atomicOr(&kmask[j >> 5], 1u << (j & 31));
       }
-      if (lane == 0 && a.col_idx[re - 1] != i) bad = true;
+      if (lane == 0 && a.col_idx[re - 1] != I) bad = true;
       if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
       __syncwarp();
       if (lane == 0) {
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(384, 1)
         int p = 0;
         for (int jt = 0; jt < n_tiles && !*abort_flag; ++jt) {
           int j = -1;
-          if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), i);
+          if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), I);
           bool stop = false;
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
@@ -264,17 +266,17 @@ __global__ void __launch_bounds__(384, 1)
             if (j < 0) {
               const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
               for (int c = 0; c < C::DCH; ++c)
-                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.blk_off[r] + jt * BN);
+                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_blk_off[r] + jt * BN);
             } else if (a.page_table == nullptr) {
               const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
               for (int c = 0; c < C::DCH; ++c)
-                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.tok_off[r] + j * BN);
+                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_tok_off[r] + j * BN);
             } else {
               const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
               const int PR = min(BN, a.page_size);
               for (int sb = 0; sb < BN / PR; ++sb) {
                 int t = j * BN + sb * PR;
-                if (t >= L) t = (L - 1) - ((L - 1) % PR);  // past the end: reload the last rows (masked)
+                if (t >= Lk) t = (Lk - 1) - ((Lk - 1) % PR);  // past the end: reload the last rows (masked)
                 int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + t / a.page_size];
                 if (page < 0 || page >= a.num_pages) {
                   set_status(a.status, FP2_DEV_PAGE_OOB);
@@ -420,7 +422,7 @@ __global__ void __launch_bounds__(384, 1)
         if (jt < n_virt) {
   #pragma unroll
           for (int c = 0; c < BN / 32; ++c) {
-            const uint32_t word = pruned_word(kmask, jt * BN + c * 32, i);
+            const uint32_t word = pruned_word(kmask, jt * BN + c * 32, I);
   #pragma unroll
             for (int e = 0; e < 32; ++e)
               xs[c * 32 + e] = ((word >> e) & 1u) ? __uint_as_float(v[c * 32 + e]) + bias_raw : -CUDART_INF_F;
@@ -559,8 +561,7 @@ __global__ void __launch_bounds__(384, 1)
 template <int DT, int D, int BN>
 static cudaError_t launch_one(const AttnArgs& a, const Fp2Plan& P, int64_t items, cudaStream_t stream) {
   using C = AttnCfg<DT, D, BN>;
-  cudaError_t e = cudaFuncSetAttribute(attention_kernel<DT, D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::SMEM_BYTES);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(attention_kernel<DT, D, BN>), C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   attention_kernel<DT, D, BN><<<static_cast<unsigned>(items), 384, C::SMEM_BYTES, stream>>>(a, P);
   return cudaGetLastError();

@@ -24,24 +24,26 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
   extern __shared__ __align__(16) float smem[];
   int r, it, g;
   if (!map_heavy_first(P, a.TI, a.Hkv, blockIdx.x, r, it, g)) return;
-  const int N = P.nblk[r], L = P.len[r];
+  // Query block i of the sequence (or chunk) is absolute key block I = pre + i.
+  const int N = P.nblk[r], L = P.len[r], pre = P.pre_blk[r];
   const int G = a.G;
   const int i0 = it * a.TI, i1 = min(N, i0 + a.TI);
   const int nI = i1 - i0, rows = nI * G;
-  const int bo = P.blk_off[r];
+  const int bo = P.blk_off[r], kbo = P.k_blk_off[r];
+  const int J1 = pre + i1;  // key blocks [0, J1) are visible to some row of the tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool dense = a.dense_all || L < a.min_sparse_len;
 
   if (dense) {  // every causal block kept
     for (int ii = warp; ii < nI; ii += 8) {
-      const int i = i0 + ii;
+      const int i = i0 + ii, I = pre + i;
       const int64_t row = static_cast<int64_t>(bo + i) * a.Hkv + g;
-      const int nw = (i + 32) / 32;
+      const int nw = (I + 32) / 32;
       for (int w = lane; w < nw; w += 32) {
-        const int nbits = min(32, i + 1 - 32 * w);
+        const int nbits = min(32, I + 1 - 32 * w);
         a.bitmask[row * a.W + w] = nbits == 32 ? 0xFFFFFFFFu : ((1u << nbits) - 1u);
       }
-      if (lane == 0) a.counts[row] = i + 1;
+      if (lane == 0) a.counts[row] = I + 1;
     }
     return;
   }
@@ -59,13 +61,13 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
         a.qbar)[(static_cast<int64_t>(bo + i0 + ii) * a.Hq + g * G + hl) * (D / 4) + c4];
   }
 
-  for (int j0 = 0; j0 < i1; j0 += kJC) {
+  for (int j0 = 0; j0 < J1; j0 += kJC) {
     __syncthreads();
     for (int idx = tid; idx < kJC * (D / 4); idx += 256) {
       const int jj = idx / (D / 4), c4 = idx % (D / 4);
       const int j = j0 + jj;
       float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < i1) val = reinterpret_cast<const float4*>(a.kbar)[(static_cast<int64_t>(bo + j) * a.Hkv + g) * (D / 4) + c4];
+      if (j < J1) val = reinterpret_cast<const float4*>(a.kbar)[(static_cast<int64_t>(kbo + j) * a.Hkv + g) * (D / 4) + c4];
       *reinterpret_cast<float4*>(&ks[jj * KS + c4 * 4]) = val;
     }
     __syncthreads();
@@ -88,16 +90,16 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int row = warp + 8 * u;
-      if (row < rows && j0 + lane < i1) sc[row * a.SP + j0 + lane] = acc[u] * a.scale;
+      if (row < rows && j0 + lane < J1) sc[row * a.SP + j0 + lane] = acc[u] * a.scale;
     }
   }
   __syncthreads();
 
   // Row max over every causal key block (forced ones included), then the threshold.
   for (int row = warp; row < rows; row += 8) {
-    const int i = i0 + row / G;
+    const int I = pre + i0 + row / G;
     float m = -CUDART_INF_F;
-    for (int j = lane; j <= i; j += 32) m = fmaxf(m, sc[row * a.SP + j]);
+    for (int j = lane; j <= I; j += 32) m = fmaxf(m, sc[row * a.SP + j]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if (lane == 0) thr[row] = m + a.ln_alpha;
@@ -106,16 +108,16 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
 
   const int win = max(a.window, 1);
   for (int ii = warp; ii < nI; ii += 8) {
-    const int i = i0 + ii;
+    const int i = i0 + ii, I = pre + i;
     const int64_t row_id = static_cast<int64_t>(bo + i) * a.Hkv + g;
-    const int nw = (i + 32) / 32;
+    const int nw = (I + 32) / 32;
     const bool last_rows = i >= N - a.last_n;
     int cnt = 0;
     for (int w = 0; w < nw; ++w) {
       const int j = w * 32 + lane;
       bool keep = false;
-      if (j <= i) {
-        keep = last_rows || (j < a.sink) || (j > i - win);
+      if (j <= I) {
+        keep = last_rows || (j < a.sink) || (j > I - win);
         for (int hl = 0; hl < G && !keep; ++hl) keep = sc[(ii * G + hl) * a.SP + j] >= thr[ii * G + hl];
       }
       const uint32_t bits = __ballot_sync(0xFFFFFFFFu, keep);
@@ -174,8 +176,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(const uint32_t* __restrict
   if (row >= rows) return;
   const int b = static_cast<int>(row / Hkv);
   const int r = seq_of_block(P, b);
-  const int i = b - P.blk_off[r];
-  const int nw = (i + 32) / 32;
+  const int I = P.pre_blk[r] + (b - P.blk_off[r]);  // absolute key block of the row's query block
+  const int nw = (I + 32) / 32;
   const int base = row_ptr[row];
   if (row_ptr[row + 1] > capacity) return;
   int prefix = 0;
@@ -209,11 +211,11 @@ cudaError_t launch_discover(const DiscArgs& a, const Fp2Plan& P, int64_t items, 
   const size_t smem = discover_smem_bytes(a.D, a.G, a.TI, a.SP);
   cudaError_t e;
   if (a.D == 64) {
-    e = cudaFuncSetAttribute(discover_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = ensure_dynamic_smem(reinterpret_cast<const void*>(discover_kernel<64>), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     discover_kernel<64><<<static_cast<unsigned>(items), 256, smem, stream>>>(a, P);
   } else {
-    e = cudaFuncSetAttribute(discover_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    e = ensure_dynamic_smem(reinterpret_cast<const void*>(discover_kernel<128>), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     discover_kernel<128><<<static_cast<unsigned>(items), 256, smem, stream>>>(a, P);
   }

@@ -7,8 +7,10 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "../../include/fp2.h"
 #include "fp2_kernels.h"
@@ -35,7 +37,7 @@ int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : (t == FP2_BF16 ? 2 : 1); 
 struct Ctx {
   Fp2Plan plan;
   int elt = 0, G = 0, W = 0;
-  int64_t T = 0, total_blocks = 0, rows = 0, cap = 0;
+  int64_t T = 0, Tk = 0, total_blocks = 0, total_k_blocks = 0, rows = 0, cap = 0;
   float scale = 0.f;
   fp2_workspace ws{};
   size_t off_bitmask = 0, off_counts = 0;  // inside scratch
@@ -76,38 +78,52 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   Fp2Plan& P = c.plan;
   std::memset(&P, 0, sizeof(P));
   P.num_seqs = p->num_seqs;
-  int64_t T = 0, blocks = 0, cap = 0;
-  int max_nblk = 0;
+  int64_t T = 0, Tk = 0, blocks = 0, kblocks = 0, cap = 0;
+  int max_nblk = 0, max_k_nblk = 0;
   for (int r = 0; r < p->num_seqs; ++r) {
     const int64_t Lq = static_cast<int64_t>(cq[r + 1]) - cq[r];
     const int64_t Lk = static_cast<int64_t>(ck[r + 1]) - ck[r];
     if (Lq < 0 || Lk < 0) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing");
-    if (Lq != Lk || cq[r] != ck[r])
-      return fail(FP2_ERR_UNSUPPORTED, "q_len != kv_len (chunked prefill) is not supported");
+    if (Lk < Lq) return fail(FP2_ERR_INVALID_ARG, "kv_len must be >= q_len for every sequence");
+    if ((Lk - Lq) % B != 0)
+      return fail(FP2_ERR_UNSUPPORTED, "a query chunk must start on a block boundary (kv_len - q_len % B != 0)");
     const int64_t N = (Lq + B - 1) / B;
-    if (N > FP2_MAX_BLOCKS) return fail(FP2_ERR_UNSUPPORTED, "a sequence has more than FP2_MAX_BLOCKS blocks");
+    const int64_t pre = (Lk - Lq) / B;
+    const int64_t Nk = pre + N;
+    if (Nk > FP2_MAX_BLOCKS) return fail(FP2_ERR_UNSUPPORTED, "a sequence has more than FP2_MAX_BLOCKS key blocks");
     P.tok_off[r] = cq[r];
     P.len[r] = static_cast<int32_t>(Lq);
     P.blk_off[r] = static_cast<int32_t>(blocks);
     P.nblk[r] = static_cast<int32_t>(N);
+    P.k_tok_off[r] = ck[r];
+    P.k_blk_off[r] = static_cast<int32_t>(kblocks);
+    P.pre_blk[r] = static_cast<int32_t>(pre);
     T += Lq;
+    Tk += Lk;
     blocks += N;
-    cap += static_cast<int64_t>(Hkv) * N * (N + 1) / 2;
+    kblocks += Nk;
+    cap += static_cast<int64_t>(Hkv) * (N * pre + N * (N + 1) / 2);  // sum_i (pre + i + 1)
     max_nblk = std::max<int>(max_nblk, static_cast<int>(N));
+    max_k_nblk = std::max<int>(max_k_nblk, static_cast<int>(Nk));
   }
-  if (T != cq[p->num_seqs]) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens inconsistent");
-  if (T >= (int64_t(1) << 31) || cap >= (int64_t(1) << 31) || blocks * Hkv >= (int64_t(1) << 31))
+  if (T != cq[p->num_seqs] || Tk != ck[p->num_seqs]) return fail(FP2_ERR_INVALID_ARG, "cu_seqlens inconsistent");
+  if (Tk >= (int64_t(1) << 31) || cap >= (int64_t(1) << 31) || kblocks * Hkv >= (int64_t(1) << 31))
     return fail(FP2_ERR_UNSUPPORTED, "problem too large for 32-bit token / index offsets");
   P.total_tokens = static_cast<int32_t>(T);
   P.total_blocks = static_cast<int32_t>(blocks);
+  P.total_k_tokens = static_cast<int32_t>(Tk);
+  P.total_k_blocks = static_cast<int32_t>(kblocks);
   P.max_nblk = max_nblk;
+  P.max_k_nblk = max_k_nblk;
   for (int r = 0; r < p->num_seqs; ++r) P.sorted[r] = static_cast<int16_t>(r);
   std::stable_sort(P.sorted, P.sorted + p->num_seqs, [&](int16_t x, int16_t y) { return P.nblk[x] > P.nblk[y]; });
   c.T = T;
+  c.Tk = Tk;
   c.total_blocks = blocks;
+  c.total_k_blocks = kblocks;
   c.rows = blocks * Hkv;
   c.cap = cap;
-  c.W = std::max(1, (max_nblk + 31) / 32);
+  c.W = std::max(1, (max_k_nblk + 31) / 32);
   c.scale = p->softmax_scale > 0.f ? p->softmax_scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
 
   // Tensors (only checked when there is data to read).
@@ -125,20 +141,22 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
       if (p->num_pages <= 0 || static_cast<int64_t>(p->num_pages) * ps >= (int64_t(1) << 31))
         return fail(FP2_ERR_INVALID_ARG, "num_pages out of range");
       for (int r = 0; r < p->num_seqs; ++r)
-        if ((P.len[r] + ps - 1) / ps > p->max_pages_per_seq)
+        if ((P.pre_blk[r] * B + P.len[r] + ps - 1) / ps > p->max_pages_per_seq)
           return fail(FP2_ERR_INVALID_ARG, "max_pages_per_seq too small for a sequence");
     }
   }
 
   fp2_workspace& w = c.ws;
   w.total_tokens = T;
-  w.total_blocks = blocks;
+  w.total_kv_tokens = Tk;
+  w.total_q_blocks = blocks;
+  w.total_kv_blocks = kblocks;
   w.index_rows = c.rows;
   w.col_capacity = cap;
   w.qbar_bytes = static_cast<size_t>(blocks) * Hq * D * 4;
-  w.kbar_bytes = static_cast<size_t>(blocks) * Hkv * D * 4;
+  w.kbar_bytes = static_cast<size_t>(kblocks) * Hkv * D * 4;
   w.vbar_bytes = w.kbar_bytes;
-  w.kbar_mma_bytes = static_cast<size_t>(blocks) * Hkv * D * c.elt;
+  w.kbar_mma_bytes = static_cast<size_t>(kblocks) * Hkv * D * c.elt;
   w.vbar_mma_bytes = w.kbar_mma_bytes;
   w.row_ptr_bytes = static_cast<size_t>(c.rows + 1) * 4;
   w.col_idx_bytes = static_cast<size_t>(std::max<int64_t>(cap, 1)) * 4;
@@ -255,6 +273,7 @@ fp2_status run_pool(const fp2_problem* p, const fp2_sparse_params* s, const Ctx&
   a.vbar = pl->vbar;
   a.kbar_mma = pl->kbar_mma;
   a.vbar_mma = pl->vbar_mma;
+  a.kv_prefix_pooled = p->kv_prefix_pooled ? 1 : 0;
   a.status = status_ptr(scratch);
   const cudaError_t e = fp2::launch_pool(p->dtype, a, c.plan, st);
   return e == cudaSuccess ? FP2_OK : cuda_fail(e, "pool kernel launch");
@@ -276,7 +295,7 @@ fp2_status run_discover(const fp2_problem* p, const fp2_sparse_params* s, const 
   a.window = s->window_blocks;
   a.last_n = s->last_n_blocks;
   a.min_sparse_len = s->min_sparse_len;
-  a.SP = std::max(32, (c.plan.max_nblk + 31) / 32 * 32);
+  a.SP = std::max(32, (c.plan.max_k_nblk + 31) / 32 * 32);
   // Largest tile of query blocks whose scores fit in shared memory (TI * G <= 32 rows).
   int TI = std::max(1, 32 / c.G);
   while (TI > 1 && fp2::discover_smem_bytes(a.D, c.G, TI, a.SP) > 200 * 1024) --TI;
@@ -304,7 +323,7 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   fp2_status st2;
   const bool paged = p->page_table != nullptr;
   if ((st2 = encode_3d(&a.tm_q, p->dtype, p->q, D, p->num_q_heads, c.T, p->q_stride_tok, B)) != FP2_OK) return st2;
-  const int64_t kv_rows = paged ? static_cast<int64_t>(p->num_pages) * p->page_size : c.T;
+  const int64_t kv_rows = paged ? static_cast<int64_t>(p->num_pages) * p->page_size : c.Tk;
   const int kv_box = paged ? std::min(B, p->page_size) : B;
   if ((st2 = encode_3d(&a.tm_k, p->dtype, p->k, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box)) != FP2_OK)
     return st2;
@@ -312,9 +331,9 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   if ((st2 = encode_3d(&a.tm_v, p->dtype, p->v, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box, v32)) != FP2_OK)
     return st2;
   const int64_t hd = static_cast<int64_t>(p->num_kv_heads) * D;
-  if ((st2 = encode_3d(&a.tm_kb, p->dtype, pl->kbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B)) != FP2_OK)
+  if ((st2 = encode_3d(&a.tm_kb, p->dtype, pl->kbar_mma, D, p->num_kv_heads, c.total_k_blocks, hd, B)) != FP2_OK)
     return st2;
-  if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_blocks, hd, B, v32)) != FP2_OK)
+  if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_k_blocks, hd, B, v32)) != FP2_OK)
     return st2;
   a.row_ptr = ix->row_ptr;
   a.col_idx = ix->col_idx;
@@ -349,6 +368,24 @@ fp2_status clear_status(void* scratch, cudaStream_t st) {
 }
 
 }  // namespace
+
+namespace fp2 {
+
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> granted;  // (kernel, device) -> bytes
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int& have = granted[{kernel, dev}];
+  if (have >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
+
+}  // namespace fp2
 
 // Used by fp2_noalloc.cu only: discovery into a caller-supplied scratch region of a fixed capacity,
 // optionally copying the device status word to status_dev afterwards.

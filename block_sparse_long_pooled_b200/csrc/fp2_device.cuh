@@ -48,9 +48,17 @@ FP2_DEVICE bool map_heavy_first(const Fp2Plan& P, int tile, int width, long long
   return false;
 }
 
+// Sequence of query block b.
 FP2_DEVICE int seq_of_block(const Fp2Plan& P, int b) {
   int r = 0;
   while (r + 1 < P.num_seqs && P.blk_off[r + 1] <= b) ++r;
+  return r;
+}
+
+// Sequence of key block b.
+FP2_DEVICE int seq_of_key_block(const Fp2Plan& P, int b) {
+  int r = 0;
+  while (r + 1 < P.num_seqs && P.k_blk_off[r + 1] <= b) ++r;
   return r;
 }
 

@@ -23,6 +23,7 @@ struct PoolArgs {
   float* vbar;
   void* kbar_mma;
   void* vbar_mma;
+  int kv_prefix_pooled;  // skip K/V of prefix blocks (already pooled)
   uint32_t* status;
 };
 
@@ -64,6 +65,11 @@ struct AttnArgs {
   int total_tokens;
   uint32_t* status;
 };
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device.  The
+// attribute call is made only when the limit grows (it is slow enough to starve the GPU when a
+// caller issues many short launches, e.g. one per prefill chunk).
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
 
 cudaError_t launch_pool(int dtype, const PoolArgs& a, const Fp2Plan& P, cudaStream_t stream);
 size_t discover_smem_bytes(int D, int G, int TI, int SP);

@@ -63,15 +63,19 @@ FP2_DEVICE void accumulate(const uint4& v, float* acc) {
   }
 }
 
+// One CTA per key block b (absolute block J of sequence r).  Its K and V rows are pooled into
+// kbar/vbar row b (skipped for prefix blocks when they are already pooled); when J lies in the
+// query chunk its Q rows are pooled into qbar row blk_off[r] + (J - pre_blk[r]).
 template <int DT>
 __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Plan P) {
   constexpr int VEC = 16 / Elt<DT>::kBytes;  // elements per 16-byte vector
   const int b = blockIdx.x;
-  const int r = seq_of_block(P, b);
-  const int i = b - P.blk_off[r];
-  const int L = P.len[r];
-  const int t0 = i * a.B;
-  const int n = min(a.B, L - t0);
+  const int r = seq_of_key_block(P, b);
+  const int J = b - P.k_blk_off[r];
+  const int pre = P.pre_blk[r];
+  const int Lk = pre * a.B + P.len[r];
+  const int t0 = J * a.B;
+  const int n = min(a.B, Lk - t0);
   const int VQ = a.Hq * a.D / VEC, VK = a.Hkv * a.D / VEC;
   const int vid = blockIdx.y * blockDim.x + threadIdx.x;
   if (vid >= VQ + 2 * VK || n <= 0) return;
@@ -80,6 +84,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Pl
   if (vid < VQ) {
     which = 0;
     col = vid * VEC;
+    if (J < pre) return;  // no query rows in prefix blocks
   } else if (vid < VQ + VK) {
     which = 1;
     col = (vid - VQ) * VEC;
@@ -87,10 +92,13 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Pl
     which = 2;
     col = (vid - VQ - VK) * VEC;
   }
+  if (which != 0 && a.kv_prefix_pooled && J < pre) return;
   const char* base = static_cast<const char*>(which == 0 ? a.q : (which == 1 ? a.k : a.v));
   const int64_t stride = which == 0 ? a.q_stride : a.kv_stride;
   const bool paged = (which != 0) && (a.page_table != nullptr);
-  const int64_t tok_base = P.tok_off[r] + t0;
+  const int64_t tok_base = which == 0 ? static_cast<int64_t>(P.tok_off[r]) + (J - pre) * a.B
+                                      : static_cast<int64_t>(P.k_tok_off[r]) + t0;
+  const int out_row = which == 0 ? P.blk_off[r] + (J - pre) : b;
 
   float acc[VEC];
 #pragma unroll
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Pl
 
   const int H = which == 0 ? a.Hq : a.Hkv;
   float* dst = which == 0 ? a.qbar : (which == 1 ? a.kbar : a.vbar);
-  float4* d4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(b) * H * a.D + col);
+  float4* d4 = reinterpret_cast<float4*>(dst + static_cast<int64_t>(out_row) * H * a.D + col);
 #pragma unroll
   for (int e = 0; e < VEC / 4; ++e)
     d4[e] = make_float4(mean_raw[4 * e] * descale, mean_raw[4 * e + 1] * descale, mean_raw[4 * e + 2] * descale,
@@ -152,7 +160,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Pl
       for (int e = 0; e < 4; ++e)
         ow[e] = pack_e4m3x4(mean_raw[4 * e], mean_raw[4 * e + 1], mean_raw[4 * e + 2], mean_raw[4 * e + 3]);
     }
-    *reinterpret_cast<uint4*>(nb + (static_cast<int64_t>(b) * H * a.D + col) * Elt<DT>::kBytes) = out;
+    *reinterpret_cast<uint4*>(nb + (static_cast<int64_t>(out_row) * H * a.D + col) * Elt<DT>::kBytes) = out;
   }
 }
 
@@ -160,7 +168,7 @@ cudaError_t launch_pool(int dtype, const PoolArgs& a, const Fp2Plan& P, cudaStre
   const int elt = dtype == FP2_F32 ? 4 : (dtype == FP2_BF16 ? 2 : 1);
   const int vec = 16 / elt;
   const int nvec = (a.Hq + 2 * a.Hkv) * a.D / vec;
-  dim3 grid(P.total_blocks, (nvec + 255) / 256);
+  dim3 grid(P.total_k_blocks, (nvec + 255) / 256);
   if (dtype == FP2_F32)
     pool_kernel<0><<<grid, 256, 0, stream>>>(a, P);
   else if (dtype == FP2_BF16)

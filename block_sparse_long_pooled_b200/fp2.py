@@ -44,6 +44,7 @@ class fp2_problem(ctypes.Structure):
         ("q_stride_tok", ctypes.c_int64), ("kv_stride_tok", ctypes.c_int64),
         ("page_table", ctypes.c_void_p),
         ("page_size", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+        ("kv_prefix_pooled", ctypes.c_int32),
     ]
 
 
@@ -66,8 +67,8 @@ class fp2_index(ctypes.Structure):
 
 class fp2_workspace(ctypes.Structure):
     _fields_ = [
-        ("total_tokens", ctypes.c_int64), ("total_blocks", ctypes.c_int64), ("index_rows", ctypes.c_int64),
-        ("col_capacity", ctypes.c_int64),
+        ("total_tokens", ctypes.c_int64), ("total_kv_tokens", ctypes.c_int64), ("total_q_blocks", ctypes.c_int64),
+        ("total_kv_blocks", ctypes.c_int64), ("index_rows", ctypes.c_int64), ("col_capacity", ctypes.c_int64),
         ("qbar_bytes", ctypes.c_size_t), ("kbar_bytes", ctypes.c_size_t), ("vbar_bytes", ctypes.c_size_t),
         ("kbar_mma_bytes", ctypes.c_size_t), ("vbar_mma_bytes", ctypes.c_size_t),
         ("row_ptr_bytes", ctypes.c_size_t), ("col_idx_bytes", ctypes.c_size_t),
@@ -136,6 +137,7 @@ class Problem:
     struct: fp2_problem
     cu_seqlens: np.ndarray
     keep: tuple
+    cu_seqlens_k: Optional[np.ndarray] = None
 
 
 def _dtype_code(t) -> int:
@@ -146,14 +148,19 @@ def _dtype_code(t) -> int:
 
 def make_problem(q, k, v, cu_seqlens, num_kv_heads: int, q_descale: float = 1.0, k_descale: float = 1.0,
                  v_descale: float = 1.0, softmax_scale: float = 0.0, page_table=None,
-                 num_pages: int = 0) -> Problem:
-    """q: [T, Hq, d]; k, v: [T, Hkv, d] or a paged cache [P, page_size, Hkv, d] with page_table
-    [num_seqs, max_pages] (int32, device).  cu_seqlens: host int sequence [num_seqs + 1]."""
+                 num_pages: int = 0, cu_seqlens_k=None, kv_prefix_pooled: bool = False) -> Problem:
+    """q: [T, Hq, d]; k, v: [Tk, Hkv, d] or a paged cache [P, page_size, Hkv, d] with page_table
+    [num_seqs, max_pages] (int32, device).  cu_seqlens: host int sequence [num_seqs + 1] of query
+    offsets; cu_seqlens_k: key offsets when the queries are chunks at the end of their sequences
+    (chunked prefill), else None.  kv_prefix_pooled: the pooled prefix K/V blocks are already in
+    the pooled buffers (see include/fp2.h)."""
     cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+    cuk = None if cu_seqlens_k is None else np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int32))
     s = fp2_problem()
     s.num_seqs = len(cu) - 1
     s.cu_seqlens_q_host = cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
-    s.cu_seqlens_k_host = s.cu_seqlens_q_host
+    s.cu_seqlens_k_host = s.cu_seqlens_q_host if cuk is None else cuk.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    s.kv_prefix_pooled = 1 if kv_prefix_pooled else 0
     s.num_q_heads = q.shape[1]
     s.num_kv_heads = num_kv_heads
     s.head_dim = q.shape[2]
@@ -171,7 +178,7 @@ def make_problem(q, k, v, cu_seqlens, num_kv_heads: int, q_descale: float = 1.0,
     else:
         s.kv_stride_tok = k.stride(0)
         s.page_table = None
-    return Problem(struct=s, cu_seqlens=cu, keep=(q, k, v, page_table))
+    return Problem(struct=s, cu_seqlens=cu, keep=(q, k, v, page_table), cu_seqlens_k=cuk)
 
 
 def make_params(block_size: int, alpha: float = 0.1, sink_blocks: int = 2, window_blocks: int = 4,
@@ -243,14 +250,14 @@ def alloc_pooled(ws: fp2_workspace, problem: Problem, device):
     """Device buffers for fp2_pooled, as torch tensors; returns (struct, dict of tensors)."""
     import torch
     s = problem.struct
-    nb, Hq, Hkv, D = ws.total_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim
+    nq, nk, Hq, Hkv, D = ws.total_q_blocks, ws.total_kv_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim
     mma_dtype = {FP2_F32: torch.float32, FP2_BF16: torch.bfloat16, FP2_E4M3: torch.uint8}[s.dtype]
     t = {
-        "qbar": torch.empty((nb, Hq, D), dtype=torch.float32, device=device),
-        "kbar": torch.empty((nb, Hkv, D), dtype=torch.float32, device=device),
-        "vbar": torch.empty((nb, Hkv, D), dtype=torch.float32, device=device),
-        "kbar_mma": torch.empty((nb, Hkv, D), dtype=mma_dtype, device=device),
-        "vbar_mma": torch.empty((nb, Hkv, D), dtype=mma_dtype, device=device),
+        "qbar": torch.empty((nq, Hq, D), dtype=torch.float32, device=device),
+        "kbar": torch.empty((nk, Hkv, D), dtype=torch.float32, device=device),
+        "vbar": torch.empty((nk, Hkv, D), dtype=torch.float32, device=device),
+        "kbar_mma": torch.empty((nk, Hkv, D), dtype=mma_dtype, device=device),
+        "vbar_mma": torch.empty((nk, Hkv, D), dtype=mma_dtype, device=device),
     }
     st = fp2_pooled(*(_ptr(t[k]) for k in ("qbar", "kbar", "vbar", "kbar_mma", "vbar_mma")))
     return st, t

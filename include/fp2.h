@@ -44,8 +44,15 @@
  *     [num_seqs, max_pages_per_seq] (device memory).
  *   - Supported: head_dim 64 or 128 (F32 and E4M3 inputs need 64 and 128
  *     respectively), block_size 64 or 128, page_size a power of two >= 16,
- *     Hq % Hkv == 0, up to FP2_MAX_SEQS sequences and FP2_MAX_BLOCKS blocks
- *     per sequence, q_len == kv_len for every sequence.
+ *     Hq % Hkv == 0, up to FP2_MAX_SEQS sequences and FP2_MAX_BLOCKS key blocks
+ *     per sequence.
+ *   - Chunked prefill (paper page, Table 6; ResearchPod: discovery re-runs per
+ *     chunk): a sequence's queries may be a chunk of its last q_len <= kv_len
+ *     tokens, aligned bottom-right (chunk token t is at absolute position
+ *     kv_len - q_len + t); kv_len - q_len must be a multiple of block_size, so
+ *     chunk block i is absolute key block I = (kv_len - q_len) / B + i, which is
+ *     what causality, the diagonal and the window refer to; last_n_blocks and
+ *     min_sparse_len refer to the chunk's queries.
  */
 #ifndef FP2_H_
 #define FP2_H_
@@ -89,8 +96,9 @@ typedef void* fp2_stream_t;
 
 typedef struct {
   int32_t num_seqs;
-  const int32_t* cu_seqlens_q_host;  /* HOST [num_seqs+1], token offsets of each sequence in Q */
-  const int32_t* cu_seqlens_k_host;  /* HOST [num_seqs+1]; must equal cu_seqlens_q_host (q_len == kv_len) */
+  const int32_t* cu_seqlens_q_host;  /* HOST [num_seqs+1], token offsets of each sequence's queries in Q */
+  const int32_t* cu_seqlens_k_host;  /* HOST [num_seqs+1], token offsets of each sequence's keys in K/V
+                                        (NULL = same as cu_seqlens_q_host); kv_len >= q_len */
   int32_t num_q_heads, num_kv_heads, head_dim;
   fp2_dtype dtype;                   /* storage type of Q, K, V (and of the MMA operands) */
   float q_descale, k_descale, v_descale;  /* value = stored * descale; 1.0 unless E4M3 */
@@ -102,6 +110,12 @@ typedef struct {
   int64_t kv_stride_tok;             /* elements between consecutive tokens of K/V (>= Hkv*d) */
   const int32_t* page_table;         /* device [num_seqs, max_pages_per_seq] or NULL for contiguous K/V */
   int32_t page_size, max_pages_per_seq, num_pages;
+  int32_t kv_prefix_pooled;          /* nonzero: the pooled kbar/vbar (and MMA copies) of every sequence's
+                                        prefix key blocks (those before its query chunk) are already in the
+                                        pooled buffers at their indices, e.g. from the previous chunk's
+                                        fp2_pool, so fp2_pool pools only the chunk's key blocks.  Valid when
+                                        those indices did not move (a single sequence, or earlier sequences
+                                        of the batch unchanged). */
 } fp2_problem;
 
 typedef struct {
@@ -116,16 +130,16 @@ typedef struct {
 
 /* Pooled block statistics (caller-owned device buffers). */
 typedef struct {
-  float* qbar;     /* [total_blocks, Hq, d] f32 block means of Q (dequantised) */
-  float* kbar;     /* [total_blocks, Hkv, d] f32 */
-  float* vbar;     /* [total_blocks, Hkv, d] f32 */
-  void* kbar_mma;  /* [total_blocks, Hkv, d] in dtype: the kbar operand of the correction MMA
+  float* qbar;     /* [total_q_blocks, Hq, d] f32 block means of Q (dequantised) */
+  float* kbar;     /* [total_kv_blocks, Hkv, d] f32 */
+  float* vbar;     /* [total_kv_blocks, Hkv, d] f32 */
+  void* kbar_mma;  /* [total_kv_blocks, Hkv, d] in dtype: the kbar operand of the correction MMA
                       (E4M3: mean of the stored values, rounded to e4m3, same descale as K) */
-  void* vbar_mma;  /* [total_blocks, Hkv, d] in dtype, likewise for V */
+  void* vbar_mma;  /* [total_kv_blocks, Hkv, d] in dtype, likewise for V */
 } fp2_pooled;
 
-/* CSR index of kept key blocks: row = (block_offset_r + i) * Hkv + g, columns are
- * sequence-local key-block ids in ascending order. */
+/* CSR index of kept key blocks: row = (q_block_offset_r + i) * Hkv + g for query block i of
+ * sequence r, columns are the sequence's absolute key-block ids in ascending order. */
 typedef struct {
   int32_t* row_ptr;      /* device [index_rows + 1] */
   int32_t* col_idx;      /* device [col_capacity] */
@@ -134,10 +148,12 @@ typedef struct {
 
 /* Sizes for one problem; every *_bytes figure is a byte count of one buffer. */
 typedef struct {
-  int64_t total_tokens;          /* T */
-  int64_t total_blocks;          /* sum_r ceil(L_r / B) */
-  int64_t index_rows;            /* total_blocks * Hkv */
-  int64_t col_capacity;          /* causal worst case: sum_r Hkv N_r (N_r + 1) / 2 */
+  int64_t total_tokens;          /* query tokens T */
+  int64_t total_kv_tokens;       /* key tokens (contiguous K/V rows) */
+  int64_t total_q_blocks;        /* sum_r ceil(q_len_r / B) */
+  int64_t total_kv_blocks;       /* sum_r ceil(kv_len_r / B) */
+  int64_t index_rows;            /* total_q_blocks * Hkv */
+  int64_t col_capacity;          /* causal worst case: sum_r Hkv sum_i (I_i + 1) */
   size_t qbar_bytes, kbar_bytes, vbar_bytes, kbar_mma_bytes, vbar_mma_bytes;
   size_t row_ptr_bytes, col_idx_bytes;
   size_t scratch_bytes;          /* scratch for fp2_pool / fp2_discover / fp2_attend */

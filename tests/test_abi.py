@@ -56,7 +56,7 @@ def test_workspace_sizes():
     prob = _problem()
     ws = fp2.fp2_workspace_query(prob, fp2.make_params(128))
     N = [8, 3]
-    assert ws.total_tokens == 1333 and ws.total_blocks == 11 and ws.index_rows == 22
+    assert ws.total_tokens == 1333 and ws.total_q_blocks == 11 and ws.total_kv_blocks == 11 and ws.index_rows == 22
     assert ws.col_capacity == sum(2 * n * (n + 1) // 2 for n in N)
     assert ws.qbar_bytes == 11 * 8 * 128 * 4 and ws.kbar_mma_bytes == 11 * 2 * 128 * 2
     assert ws.row_ptr_bytes == 23 * 4 and ws.col_idx_bytes == ws.col_capacity * 4
@@ -85,13 +85,22 @@ def test_validation_errors(kw, params, code):
     assert fp2.fp2_last_error() != ""
 
 
-def test_chunked_prefill_rejected():
-    prob = _problem()
-    ck = np.array([0, 900, 1333], dtype=np.int32)
-    prob.struct.cu_seqlens_k_host = ck.ctypes.data_as(prob.struct.cu_seqlens_k_host.__class__)
-    with pytest.raises(fp2.FP2Error) as e:
-        fp2.fp2_workspace_query(prob, fp2.make_params(128))
-    assert e.value.status == fp2.FP2_ERR_UNSUPPORTED
+def test_chunked_prefill_sizes_and_rules():
+    # queries: chunks of 1000 and 333 tokens; keys: 1000 + 256 and 333 + 512 (prefixes of 2 and 4 blocks)
+    T, Tk, Hq, Hkv, d = 1333, 2101, 8, 2, 128
+    q = torch.empty((T, Hq, d), dtype=torch.bfloat16)
+    k = torch.empty((Tk, Hkv, d), dtype=torch.bfloat16)
+    prob = fp2.make_problem(q, k, k, [0, 1000, 1333], Hkv, cu_seqlens_k=[0, 1256, 2101])
+    ws = fp2.fp2_workspace_query(prob, fp2.make_params(128))
+    assert ws.total_kv_tokens == Tk and ws.total_q_blocks == 8 + 3 and ws.total_kv_blocks == 10 + 7
+    assert ws.col_capacity == 2 * (sum(2 + i + 1 for i in range(8)) + sum(4 + i + 1 for i in range(3)))
+    assert ws.kbar_bytes == 17 * Hkv * d * 4 and ws.qbar_bytes == 11 * Hq * d * 4
+    for cuk, code in (([0, 1200, 2045], fp2.FP2_ERR_UNSUPPORTED),      # prefix 200 not a multiple of 128
+                      ([0, 900, 1745], fp2.FP2_ERR_INVALID_ARG)):      # kv_len < q_len
+        bad = fp2.make_problem(q, k, k, [0, 1000, 1333], Hkv, cu_seqlens_k=cuk)
+        with pytest.raises(fp2.FP2Error) as e:
+            fp2.fp2_workspace_query(bad, fp2.make_params(128))
+        assert e.value.status == code
 
 
 def test_scratch_too_small_rejected_before_launch():
