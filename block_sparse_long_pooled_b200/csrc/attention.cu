@@ -13,6 +13,10 @@
 // correction shares the exact path's MMAs and online softmax; kept blocks and blocks >= i
 // are masked out of the virtual tiles.  The last kept block is the diagonal (causal mask).
 //
+// KV splits: with few rows, each row's key stream can be cut into `splits` contiguous ranges of
+// equal tile count (count-balanced; paper page, Table 7); every range is a separate CTA writing a
+// normalised partial O and its LSE, merged afterwards by combine_kernel.
+//
 // Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S,
 //                    mask, online max with lazy O rescale (only when the running max grows
@@ -165,8 +169,9 @@ __global__ void __launch_bounds__(384, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int r, i, sub;
-  if (!map_heavy_first(P, 1, a.Hkv * a.parts, blockIdx.x, r, i, sub)) return;
-  const int g = sub / a.parts, part = sub % a.parts;
+  if (!map_heavy_first(P, 1, a.Hkv * a.parts * a.splits, blockIdx.x, r, i, sub)) return;
+  const int split = sub % a.splits;
+  const int g = (sub / a.splits) / a.parts, part = (sub / a.splits) % a.parts;
   const int L = P.len[r];                 // query tokens of the sequence (or chunk)
   const int I = P.pre_blk[r] + i;         // absolute key block of query block i (the diagonal)
   const int Lk = P.pre_blk[r] * BN + L;   // key tokens of the sequence
@@ -180,6 +185,10 @@ __global__ void __launch_bounds__(384, 1)
   const int npruned = I + 1 - nkept;
   const int n_virt = (a.mean_correction && npruned > 0) ? (I + BN - 1) / BN : 0;
   const int n_tiles = n_virt + nkept;
+  // Count-balanced KV split: this CTA takes key tiles [t_begin, t_end) of the row's stream.
+  const int t_begin = static_cast<int>(static_cast<long long>(n_tiles) * split / a.splits);
+  const int t_end = static_cast<int>(static_cast<long long>(n_tiles) * (split + 1) / a.splits);
+  const int n_local = t_end - t_begin;
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -206,9 +215,6 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Register split: the launch gives 384 threads x 168 registers; warpgroup 2 (producer, MMA,
-  // two idle warps) drops to 56 and the two softmax warpgroups rise to 224:
-  // 128 x 56 + 256 x 224 = 64512 = 384 x 168.
-  // Register split: the launch gives 384 threads x 168 registers; warpgroup 2 (producer, MMA,
   // two idle warps) drops to REG_LOW and the two softmax warpgroups rise to REG_HIGH, with
   // 128 * REG_LOW + 256 * REG_HIGH <= 384 * 168 (checked at compile time).
 
@@ -216,23 +222,8 @@ __global__ void __launch_bounds__(384, 1)
     setmaxnreg_dec<C::REG_LOW>();
     if (warp == 8) {
       // ---------------------------------------------------------------- producer
-      const int nw = (I + 32) / 32;
-      for (int w = lane; w < nw; w += 32) kmask[w] = 0u;
-      __syncwarp();
-      bool bad = false;
-      for (int e = lane; e < nkept; e += 32) {
-        const int j = a.col_idx[rs + e];
-        const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
-        if (j < 0 || j > I || j <= prev)
-          bad = true;
-        else
-          atomicOr(&kmask[j >> 5], 1u << (j & 31));
-      }
-      if (lane == 0 && a.col_idx[re - 1] != I) bad = true;
-      if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
-      __syncwarp();
+      // Q first (it has no dependency), then the kept-block mask while Q is in flight.
       if (lane == 0) {
-        mbar_arrive(mask_ready);
         tma_prefetch_desc(&a.tm_q);
         tma_prefetch_desc(&a.tm_k);
         tma_prefetch_desc(&a.tm_v);
@@ -250,8 +241,26 @@ __global__ void __launch_bounds__(384, 1)
                           c * C::KCH, h, tokq);
           }
         }
+      }
+      const int nw = (I + 32) / 32;
+      for (int w = lane; w < nw; w += 32) kmask[w] = 0u;
+      __syncwarp();
+      bool bad = false;
+      for (int e = lane; e < nkept; e += 32) {
+        const int j = a.col_idx[rs + e];
+        const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
+        if (j < 0 || j > I || j <= prev)
+          bad = true;
+        else
+          atomicOr(&kmask[j >> 5], 1u << (j & 31));
+      }
+      if (lane == 0 && a.col_idx[re - 1] != I) bad = true;
+      if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) set_status(a.status, FP2_DEV_INDEX_OOB);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(mask_ready);
         int p = 0;
-        for (int jt = 0; jt < n_tiles && !*abort_flag; ++jt) {
+        for (int jt = t_begin; jt < t_end && !*abort_flag; ++jt) {
           int j = -1;
           if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), I);
           bool stop = false;
@@ -340,7 +349,7 @@ __global__ void __launch_bounds__(384, 1)
         int p = 0;
         int vslot_prev = 0;
         uint32_t vaddr_prev = 0;
-        for (int jt = 0; jt < n_tiles && ok; ++jt) {
+        for (int jt = 0; jt < n_local && ok; ++jt) {  // jt: tile index within this split
           const int kslot = p % C::NSLOT;
           if (!mbar_wait(&kv_full[kslot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
           ++p;
@@ -375,7 +384,7 @@ __global__ void __launch_bounds__(384, 1)
           } else {
             umma_commit(&kv_empty[vslot]);
           }
-          if (jt == n_tiles - 1 && a.NT == 2) {
+          if (jt == n_local - 1 && a.NT == 2) {
             if (!mbar_wait(&p_full[1], jt & 1, abort_flag, a.status)) break;
             tc_fence_after();
             issue_pv(1, vaddr, jt);
@@ -405,8 +414,9 @@ __global__ void __launch_bounds__(384, 1)
       float m_run = -CUDART_INF_F, l_run = 0.f;
       bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status));
       int done_tiles = 0;
-      for (int jt = 0; jt < n_tiles && ok; ++jt) {
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jt & 1, abort_flag, a.status));
+      for (int jl = 0; jl < n_local && ok; ++jl) {
+        const int jt = t_begin + jl;  // position in the row's key stream
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jl & 1, abort_flag, a.status));
         if (!ok) break;
         tc_fence_after();
         // The whole S row of this thread, in registers.
@@ -445,7 +455,7 @@ __global__ void __launch_bounds__(384, 1)
         const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * s2;
         const float m_new = fmaxf(m_run, mt);
         const bool need = m_new > m_run + C::LAZY;
-        if (jt > 0 && __any_sync(0xFFFFFFFFu, need)) {
+        if (jl > 0 && __any_sync(0xFFFFFFFFu, need)) {
           const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
   #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -510,12 +520,40 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         mbar_arrive(&p_full[s]);
         l_run += rsum;
-        done_tiles = jt + 1;
+        done_tiles = jl + 1;
       }
-      if (ok && done_tiles == n_tiles)
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_tiles - 1) & 1, abort_flag, a.status));
+      if (ok && done_tiles == n_local && n_local > 0)
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_local - 1) & 1, abort_flag, a.status));
       tc_fence_after();
-      if (ok) {
+      if (ok && a.splits > 1) {
+        // Partial result of this split: normalised O (fp32) and its natural-log LSE, merged by
+        // combine_kernel.  A split with no key tile (or no visible key for this row) contributes
+        // O = 0 with LSE = -inf.
+        const int tok = P.tok_off[r] + i * BN + tl;
+        const bool any = n_local > 0 && l_run > 0.f;
+        const float inv = any ? a.v_descale / l_run : 0.f;
+        float* op = a.o_part + ((static_cast<int64_t>(split) * a.total_tokens + tok) * a.Hq + h) * D;
+  #pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (n_local > 0) {
+            tmem_ld32_sync(o_addr + c * 32, v);
+          } else {
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(op + c * 32);
+  #pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                   __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+          }
+        }
+        if (row_ok)
+          a.lse_part[(static_cast<int64_t>(split) * a.Hq + h) * a.total_tokens + tok] =
+              any ? (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f : -CUDART_INF_F;
+      } else if (ok) {
         const int tok = P.tok_off[r] + i * BN + tl;
         const float inv = a.v_descale / l_run;
   #pragma unroll
@@ -556,6 +594,60 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// Merge of the KV-split partials: for every (token, head), O = sum_s w_s O_s / sum_s w_s and
+// LSE = m + ln sum_s w_s with w_s = exp(LSE_s - m), m = max_s LSE_s.  One warp per row, each lane
+// owning D/32 consecutive-by-lane columns (coalesced).
+template <int D, bool F32OUT>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ o_part,
+                                                      const float* __restrict__ lse_part, int S, int T, int Hq,
+                                                      void* out, float* lse) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= static_cast<int64_t>(T) * Hq) return;
+  const int t = static_cast<int>(row / Hq), h = static_cast<int>(row % Hq);
+  float m = -CUDART_INF_F;
+  for (int s = 0; s < S; ++s) m = fmaxf(m, lse_part[(static_cast<int64_t>(s) * Hq + h) * T + t]);
+  float acc[D / 32];
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) acc[k] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float l = lse_part[(static_cast<int64_t>(s) * Hq + h) * T + t];
+    const float w = (l == -CUDART_INF_F) ? 0.f : expf(l - m);
+    wsum += w;
+    const float* src = o_part + ((static_cast<int64_t>(s) * T + t) * Hq + h) * D;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) acc[k] = fmaf(w, src[lane + 32 * k], acc[k]);
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {
+    const int64_t idx = (static_cast<int64_t>(t) * Hq + h) * D + lane + 32 * k;
+    if constexpr (F32OUT)
+      static_cast<float*>(out)[idx] = acc[k] * inv;
+    else
+      static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(acc[k] * inv);
+  }
+  if (lse != nullptr && lane == 0) lse[static_cast<int64_t>(h) * T + t] = m + logf(wsum);
+}
+
+cudaError_t launch_combine(int dtype, int D, const float* o_part, const float* lse_part, int S, int T, int Hq,
+                           void* out, float* lse, cudaStream_t stream) {
+  const int64_t rows = static_cast<int64_t>(T) * Hq;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  if (blocks == 0) return cudaSuccess;
+  const bool f32 = dtype == FP2_F32;
+  if (D == 64 && f32)
+    combine_kernel<64, true><<<blocks, 256, 0, stream>>>(o_part, lse_part, S, T, Hq, out, lse);
+  else if (D == 64)
+    combine_kernel<64, false><<<blocks, 256, 0, stream>>>(o_part, lse_part, S, T, Hq, out, lse);
+  else if (f32)
+    combine_kernel<128, true><<<blocks, 256, 0, stream>>>(o_part, lse_part, S, T, Hq, out, lse);
+  else
+    combine_kernel<128, false><<<blocks, 256, 0, stream>>>(o_part, lse_part, S, T, Hq, out, lse);
+  return cudaGetLastError();
 }
 
 template <int DT, int D, int BN>

@@ -41,6 +41,8 @@ struct Ctx {
   float scale = 0.f;
   fp2_workspace ws{};
   size_t off_bitmask = 0, off_counts = 0;  // inside scratch
+  int NT = 1, parts = 1, splits = 1;        // attention launch shape
+  size_t off_opart = 0, off_lsepart = 0;    // KV-split partials inside scratch (splits > 1)
   // fp2_prefill carve-outs (offsets after scratch_bytes)
   size_t off_qbar = 0, off_kbar = 0, off_vbar = 0, off_kbm = 0, off_vbm = 0, off_rowptr = 0, off_colidx = 0;
 };
@@ -65,6 +67,7 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   if (!(s->alpha >= 0.f && s->alpha <= 1.f)) return fail(FP2_ERR_INVALID_ARG, "alpha must be in [0, 1]");
   if (s->sink_blocks < 0 || s->window_blocks < 0 || s->last_n_blocks < 0 || s->min_sparse_len < 0)
     return fail(FP2_ERR_INVALID_ARG, "sink/window/last_n/min_sparse_len must be >= 0");
+  if (s->kv_splits < 0 || s->kv_splits > 64) return fail(FP2_ERR_INVALID_ARG, "kv_splits must be in [0, 64]");
   if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale))
     return fail(FP2_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   for (float d : {p->q_descale, p->k_descale, p->v_descale})
@@ -160,9 +163,25 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   w.vbar_mma_bytes = w.kbar_mma_bytes;
   w.row_ptr_bytes = static_cast<size_t>(c.rows + 1) * 4;
   w.col_idx_bytes = static_cast<size_t>(std::max<int64_t>(cap, 1)) * 4;
+  // Attention launch shape: M tiles of 128 packed rows, two per CTA when the group fills them.
+  const int mtiles = (c.G * B + 127) / 128;
+  c.NT = mtiles >= 2 ? 2 : 1;
+  c.parts = (mtiles + c.NT - 1) / c.NT;
+  const int64_t row_ctas = c.rows * c.parts;
+  if (s->kv_splits > 0)
+    c.splits = s->kv_splits;
+  else
+    c.splits = row_ctas >= 296 ? 1 : static_cast<int>(std::min<int64_t>(8, (296 + std::max<int64_t>(row_ctas, 1) - 1) /
+                                                                                   std::max<int64_t>(row_ctas, 1)));
   c.off_bitmask = FP2_SCRATCH_STATUS_BYTES;
   c.off_counts = c.off_bitmask + align_up(static_cast<size_t>(c.rows) * c.W * 4);
   w.scratch_bytes = c.off_counts + align_up(static_cast<size_t>(c.rows) * 4);
+  w.discover_scratch_bytes = w.scratch_bytes;
+  if (c.splits > 1) {
+    c.off_opart = w.scratch_bytes;
+    c.off_lsepart = c.off_opart + align_up(static_cast<size_t>(c.splits) * T * Hq * D * 4);
+    w.scratch_bytes = c.off_lsepart + align_up(static_cast<size_t>(c.splits) * Hq * T * 4);
+  }
   size_t o = w.scratch_bytes;
   c.off_qbar = o;   o += align_up(w.qbar_bytes);
   c.off_kbar = o;   o += align_up(w.kbar_bytes);
@@ -346,9 +365,11 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   a.Hq = p->num_q_heads;
   a.Hkv = p->num_kv_heads;
   a.G = c.G;
-  const int mtiles = (c.G * B + 127) / 128;
-  a.NT = mtiles >= 2 ? 2 : 1;
-  a.parts = (mtiles + a.NT - 1) / a.NT;
+  a.NT = c.NT;
+  a.parts = c.parts;
+  a.splits = c.splits;
+  a.o_part = c.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(scratch) + c.off_opart) : nullptr;
+  a.lse_part = c.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(scratch) + c.off_lsepart) : nullptr;
   a.sm_scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634 *
                                        static_cast<double>(p->q_descale) * static_cast<double>(p->k_descale));
   a.v_descale = p->v_descale;
@@ -356,10 +377,16 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   a.mean_correction = s->mean_correction ? 1 : 0;
   a.total_tokens = static_cast<int>(c.T);
   a.status = status_ptr(scratch);
-  const int64_t items = c.total_blocks * p->num_kv_heads * a.parts;
+  const int64_t items = c.total_blocks * p->num_kv_heads * a.parts * a.splits;
   if (items == 0) return FP2_OK;
-  const cudaError_t e = fp2::launch_attention(p->dtype, D, B, a, c.plan, items, st);
-  return e == cudaSuccess ? FP2_OK : cuda_fail(e, "attention kernel launch");
+  cudaError_t e = fp2::launch_attention(p->dtype, D, B, a, c.plan, items, st);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  if (c.splits > 1) {
+    e = fp2::launch_combine(p->dtype, D, a.o_part, a.lse_part, c.splits, static_cast<int>(c.T), p->num_q_heads, out,
+                            lse, st);
+    if (e != cudaSuccess) return cuda_fail(e, "split combine kernel launch");
+  }
+  return FP2_OK;
 }
 
 fp2_status clear_status(void* scratch, cudaStream_t st) {
@@ -399,8 +426,8 @@ fp2_status discover_fixed_scratch(const fp2_problem* problem, const fp2_sparse_p
   Ctx c;
   fp2_status s;
   if ((s = validate(problem, params, c)) != FP2_OK) return s;
-  if (c.ws.scratch_bytes > capacity)
-    return fail(FP2_ERR_UNSUPPORTED, "problem needs " + std::to_string(c.ws.scratch_bytes) +
+  if (c.ws.discover_scratch_bytes > capacity)
+    return fail(FP2_ERR_UNSUPPORTED, "problem needs " + std::to_string(c.ws.discover_scratch_bytes) +
                                          " bytes of discovery scratch; the static buffer holds " +
                                          std::to_string(capacity));
   if ((s = check_pooled(pooled, true)) != FP2_OK) return s;

@@ -63,6 +63,9 @@ struct AttnArgs {
   float log2_blk;             // log2 of a pruned block's token count
   int mean_correction;
   int total_tokens;
+  int splits;                 // KV splits per row (1 = none)
+  float* o_part;              // [splits, T, Hq, d] f32 partial outputs (splits > 1)
+  float* lse_part;            // [splits, Hq, T] f32 partial LSE (splits > 1)
   uint32_t* status;
 };
 
@@ -79,5 +82,7 @@ cudaError_t launch_discover(const DiscArgs& a, const Fp2Plan& P, int64_t items, 
 cudaError_t launch_attention(int dtype, int D, int B, const AttnArgs& a, const Fp2Plan& P, int64_t items,
                              cudaStream_t stream);
 size_t attention_smem_bytes(int dtype, int D, int B);
+cudaError_t launch_combine(int dtype, int D, const float* o_part, const float* lse_part, int S, int T, int Hq,
+                           void* out, float* lse, cudaStream_t stream);
 
 }  // namespace fp2

@@ -52,7 +52,7 @@ class fp2_sparse_params(ctypes.Structure):
     _fields_ = [
         ("block_size", ctypes.c_int32), ("alpha", ctypes.c_float), ("sink_blocks", ctypes.c_int32),
         ("window_blocks", ctypes.c_int32), ("last_n_blocks", ctypes.c_int32), ("min_sparse_len", ctypes.c_int32),
-        ("mean_correction", ctypes.c_int32),
+        ("mean_correction", ctypes.c_int32), ("kv_splits", ctypes.c_int32),
     ]
 
 
@@ -72,7 +72,8 @@ class fp2_workspace(ctypes.Structure):
         ("qbar_bytes", ctypes.c_size_t), ("kbar_bytes", ctypes.c_size_t), ("vbar_bytes", ctypes.c_size_t),
         ("kbar_mma_bytes", ctypes.c_size_t), ("vbar_mma_bytes", ctypes.c_size_t),
         ("row_ptr_bytes", ctypes.c_size_t), ("col_idx_bytes", ctypes.c_size_t),
-        ("scratch_bytes", ctypes.c_size_t), ("prefill_scratch_bytes", ctypes.c_size_t),
+        ("discover_scratch_bytes", ctypes.c_size_t), ("scratch_bytes", ctypes.c_size_t),
+        ("prefill_scratch_bytes", ctypes.c_size_t),
     ]
 
 
@@ -182,9 +183,10 @@ def make_problem(q, k, v, cu_seqlens, num_kv_heads: int, q_descale: float = 1.0,
 
 
 def make_params(block_size: int, alpha: float = 0.1, sink_blocks: int = 2, window_blocks: int = 4,
-                last_n_blocks: int = 0, min_sparse_len: int = 0, mean_correction: bool = True) -> fp2_sparse_params:
+                last_n_blocks: int = 0, min_sparse_len: int = 0, mean_correction: bool = True,
+                kv_splits: int = 0) -> fp2_sparse_params:
     return fp2_sparse_params(block_size, alpha, sink_blocks, window_blocks, last_n_blocks, min_sparse_len,
-                             1 if mean_correction else 0)
+                             1 if mean_correction else 0, kv_splits)
 
 
 # ------------------------------------------------------------------ the C entry points

@@ -126,6 +126,10 @@ typedef struct {
   int32_t last_n_blocks;    /* the last n query blocks of each sequence keep every key block */
   int32_t min_sparse_len;   /* sequences shorter than this keep every block */
   int32_t mean_correction;  /* nonzero: pruned blocks contribute their pooled term */
+  int32_t kv_splits;        /* count-balanced KV splits per row (paper page, Table 7): each row's key
+                               tiles are cut into this many equal ranges processed by separate CTAs
+                               and merged by their LSE; 1 = no split; 0 = automatic (split only when
+                               rows x packed parts < 296, into up to 8 ranges); at most 64 */
 } fp2_sparse_params;
 
 /* Pooled block statistics (caller-owned device buffers). */
@@ -156,7 +160,8 @@ typedef struct {
   int64_t col_capacity;          /* causal worst case: sum_r Hkv sum_i (I_i + 1) */
   size_t qbar_bytes, kbar_bytes, vbar_bytes, kbar_mma_bytes, vbar_mma_bytes;
   size_t row_ptr_bytes, col_idx_bytes;
-  size_t scratch_bytes;          /* scratch for fp2_pool / fp2_discover / fp2_attend */
+  size_t discover_scratch_bytes; /* the part of scratch that fp2_discover uses (status, kept bits, counts) */
+  size_t scratch_bytes;          /* scratch for fp2_pool / fp2_discover / fp2_attend (adds KV-split partials) */
   size_t prefill_scratch_bytes;  /* scratch for fp2_prefill (adds pooled and index buffers) */
 } fp2_workspace;
 
@@ -203,7 +208,7 @@ FP2_API fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_o
  * device allocator).  The paper has no counterpart: this is fp2_discover with its scratch moved into
  * a library-owned static __device__ buffer of FP2_STATIC_SCRATCH_BYTES per GPU, held until exit.
  * Inputs (pooled) and outputs (index) are still the caller's.  Returns FP2_ERR_UNSUPPORTED when the
- * problem's fp2_workspace.scratch_bytes exceeds FP2_STATIC_SCRATCH_BYTES.  Allocates nothing.  The
+ * problem's fp2_workspace.discover_scratch_bytes exceeds FP2_STATIC_SCRATCH_BYTES.  Allocates nothing.  The
  * first call on a device looks up the buffer's address (make it before any stream capture).  All
  * calls share the buffer: calls that overlap on the GPU race, so serialise them.  status_dev
  * (device pointer, or NULL) receives a copy of the FP2_DEV_* status word of this call. */

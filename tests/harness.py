@@ -78,13 +78,13 @@ def gpu_params(w: W.Workload, **over):
     return fp2.make_params(**kw)
 
 
-def run_gpu(inp: W.Inputs, external_index: Optional[tuple] = None, lse: bool = True) -> GpuRun:
+def run_gpu(inp: W.Inputs, external_index: Optional[tuple] = None, lse: bool = True, kv_splits: int = 0) -> GpuRun:
     """pool -> discover -> attend through the C ABI (attend on external_index when given)."""
     import torch
     from block_sparse_long_pooled_b200 import fp2
     dev = to_device(inp)
     prob = make_gpu_problem(inp, dev)
-    params = gpu_params(inp.workload)
+    params = gpu_params(inp.workload, kv_splits=kv_splits)
     ws = fp2.fp2_workspace_query(prob, params)
     pst, pooled = fp2.alloc_pooled(ws, prob, "cuda")
     ist, index = fp2.alloc_index(ws, "cuda")

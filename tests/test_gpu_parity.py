@@ -71,6 +71,33 @@ def test_small_full_parity(w):
         Hn.compare_attention_full(run2, inp, ora)
 
 
+SPLIT_CASES = [
+    (small("split_bf16_g4", seqlens=(1500, 600)), 2),
+    (small("split_bf16_g8_paged", num_q_heads=16, num_kv_heads=2, seqlens=(2000,), paged=True, page_size=64), 3),
+    (small("split_e4m3", dtype="e4m3", seqlens=(1800,)), 5),
+    (small("split_f32_d64_b64", dtype="f32", num_q_heads=2, num_kv_heads=2, head_dim=64, block_size=64,
+           seqlens=(1100,)), 4),
+    # few rows (one KV head, 2048 tokens): the automatic rule splits every row
+    (small("split_auto_few_rows", num_q_heads=4, num_kv_heads=1, seqlens=(2048,), sink_blocks=2, window_blocks=4), 0),
+]
+
+
+@pytest.mark.parametrize("case", SPLIT_CASES, ids=[c[0].name for c in SPLIT_CASES])
+def test_kv_splits_match_oracle(case):
+    """Count-balanced KV splits (per-range partials merged by LSE) give the oracle's output."""
+    from block_sparse_long_pooled_b200 import fp2
+    w, splits = case
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), kv_splits=splits)
+    Hn.compare_attention_full(run, inp, ora)
+    if splits == 0:
+        ws = fp2.fp2_workspace_query(run.problem, run.params)
+        one = fp2.fp2_workspace_query(run.problem, Hn.gpu_params(w, kv_splits=1))
+        assert ws.scratch_bytes > one.scratch_bytes          # partial buffers were sized: it did split
+
+
 def test_tiny_workload_end_to_end():
     """The 1K fp32 workload with its four planted needle blocks, through fp2_prefill."""
     import torch

@@ -35,7 +35,7 @@ def _index_both_ways(w):
     prob = Hn.make_gpu_problem(inp, dev)
     params = Hn.gpu_params(w)
     ws = fp2.fp2_workspace_query(prob, params)
-    assert ws.scratch_bytes <= fp2.FP2_STATIC_SCRATCH_BYTES
+    assert ws.discover_scratch_bytes <= fp2.FP2_STATIC_SCRATCH_BYTES
     pst, _ = fp2.alloc_pooled(ws, prob, "cuda")
     scratch = fp2.alloc_scratch(ws.scratch_bytes, "cuda")
     fp2.fp2_pool(prob, params, pst, scratch)
@@ -77,7 +77,7 @@ def test_static_discovery_rejects_oversized_problem():
     prob = fp2.make_problem(q, q, q, cu, 8)
     params = fp2.make_params(64)
     ws = fp2.fp2_workspace_query(prob, params)
-    assert ws.scratch_bytes > fp2.FP2_STATIC_SCRATCH_BYTES
+    assert ws.discover_scratch_bytes > fp2.FP2_STATIC_SCRATCH_BYTES
     pst = fp2.fp2_pooled(q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr())
     ix = fp2.fp2_index(q.data_ptr(), q.data_ptr(), 1)
     with pytest.raises(fp2.FP2Error) as e:
