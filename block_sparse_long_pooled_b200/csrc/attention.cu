@@ -444,15 +444,16 @@ __global__ void __launch_bounds__(384, 1)
   #pragma unroll
           for (int e = 0; e < BN; ++e) xs[e] = __uint_as_float(v[e]);
         }
-        float m4[4] = {xs[0], xs[1], xs[2], xs[3]};
+        // Row max with three-operand max, four independent chains.
+        float m4[4];
   #pragma unroll
-        for (int e = 4; e < BN; e += 4) {
-          m4[0] = fmaxf(m4[0], xs[e]);
-          m4[1] = fmaxf(m4[1], xs[e + 1]);
-          m4[2] = fmaxf(m4[2], xs[e + 2]);
-          m4[3] = fmaxf(m4[3], xs[e + 3]);
+        for (int u = 0; u < 4; ++u) m4[u] = fmaxf(xs[2 * u], xs[2 * u + 1]);
+  #pragma unroll
+        for (int e = 8; e < BN; e += 8) {
+  #pragma unroll
+          for (int u = 0; u < 4; ++u) m4[u] = fmax3(m4[u], xs[e + 2 * u], xs[e + 2 * u + 1]);
         }
-        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * s2;
+        const float mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * s2;
         const float m_new = fmaxf(m_run, mt);
         const bool need = m_new > m_run + C::LAZY;
         if (jl > 0 && __any_sync(0xFFFFFFFFu, need)) {
@@ -462,7 +463,12 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t o[32];
             tmem_ld32_sync(o_addr + c * 32, o);
   #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            for (int e = 0; e < 32; e += 2) {
+              const float2 r2 = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])),
+                                           make_float2(f, f));
+              o[e] = __float_as_uint(r2.x);
+              o[e + 1] = __float_as_uint(r2.y);
+            }
             tmem_st32(o_addr + c * 32, o);
           }
           tmem_st_wait();
@@ -473,16 +479,22 @@ __global__ void __launch_bounds__(384, 1)
         }
         // P = 2^(S*s2 - m + P_SHIFT), packed to the MMA operand type and written over S in TMEM.
         const float nmu = C::P_SHIFT - ((m_run == -CUDART_INF_F) ? 0.f : m_run);
-        float rs[2] = {0.f, 0.f};
+        // Exponent arguments x * s2 + nmu and the row sums in packed f32x2 arithmetic (pairs of
+        // adjacent scores); the same fused multiply-add as the scalar form, so P is unchanged.
+        const float2 s22 = make_float2(s2, s2), nmu2 = make_float2(nmu, nmu);
+        float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        auto exp_pair = [&](int e2) -> float2 {
+          const float2 t = __ffma2_rn(make_float2(xs[2 * e2], xs[2 * e2 + 1]), s22, nmu2);
+          const float2 p = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          acc[e2 & 1] = __fadd2_rn(acc[e2 & 1], p);
+          return p;
+        };
         if constexpr (DT == 1) {
           uint32_t pk[BN / 2];
   #pragma unroll
           for (int e = 0; e < BN / 2; ++e) {
-            const float p0 = fast_exp2(fmaf(xs[2 * e], s2, nmu));
-            const float p1 = fast_exp2(fmaf(xs[2 * e + 1], s2, nmu));
-            rs[0] += p0;
-            rs[1] += p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            const float2 p = exp_pair(e);
+            pk[e] = pack_bf16x2(p.x, p.y);
           }
   #pragma unroll
           for (int c = 0; c < BN / 64; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
@@ -493,13 +505,8 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < BN / 32; ++c) {
   #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              float q4[4];
-  #pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                q4[u] = fast_exp2(fmaf(xs[c * 32 + 4 * e + u], s2, nmu));
-                rs[u & 1] += q4[u];
-              }
-              split_e4m3x4(q4[0], q4[1], q4[2], q4[3], pk[c * 16 + e], pk[c * 16 + 8 + e]);
+              const float2 pa = exp_pair(c * 16 + 2 * e), pb = exp_pair(c * 16 + 2 * e + 1);
+              split_e4m3x4(pa.x, pa.y, pb.x, pb.y, pk[c * 16 + e], pk[c * 16 + 8 + e]);
             }
           }
   #pragma unroll
@@ -507,15 +514,15 @@ __global__ void __launch_bounds__(384, 1)
         } else {
           uint32_t pk[BN];
   #pragma unroll
-          for (int e = 0; e < BN; ++e) {
-            const float p0 = fast_exp2(fmaf(xs[e], s2, nmu));
-            rs[e & 1] += p0;
-            pk[e] = __float_as_uint(p0);
+          for (int e = 0; e < BN / 2; ++e) {
+            const float2 p = exp_pair(e);
+            pk[2 * e] = __float_as_uint(p.x);
+            pk[2 * e + 1] = __float_as_uint(p.y);
           }
   #pragma unroll
           for (int c = 0; c < BN / 32; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
         }
-        const float rsum = rs[0] + rs[1];
+        const float rsum = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[s]);

@@ -269,6 +269,13 @@ FP2_DEVICE float fast_exp2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (three-operand max.f32, sm_100).
+FP2_DEVICE float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Two floats -> packed bf16x2 (lo in the low half).
 FP2_DEVICE uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
