@@ -36,7 +36,7 @@
 namespace fp2 {
 
 #ifndef REG_LOW_T
-#define REG_LOW_T 56
+#define REG_LOW_T 80
 #endif
 
 template <int DT, int D, int BN>
@@ -309,9 +309,14 @@ __global__ void __launch_bounds__(384, 1)
       // Ping-pong order per key tile j: QK0(j), PV1(j-1), QK1(j), PV0(j).  The softmax of tile 0
       // then runs while the tensor pipe does PV1(j-1) and QK1(j), and the softmax of tile 1 while
       // it does PV0(j) and QK0(j+1), so the two softmax warpgroups alternate instead of competing.
-      if (lane == 0) {
+      // The whole warp runs this loop with warp-uniform control flow (every wait is voted) and
+      // lane 0 issues each tcgen05 instruction (the *_warp wrappers).
+      {
+        auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+          return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, a.status));
+        };
         bool ok = true;
-        for (int s = 0; s < a.NT && ok; ++s) ok = mbar_wait(&q_full[s], 0, abort_flag, a.status);
+        for (int s = 0; s < a.NT && ok; ++s) ok = wait_all(&q_full[s], 0);
         tc_fence_after();
         // Descriptors are formed once per tile; a K step only moves the start address, which is
         // the low 14 bits (address >> 4) of the descriptor and cannot carry (shared memory < 256 KB).
@@ -319,14 +324,15 @@ __global__ void __launch_bounds__(384, 1)
           const uint64_t ad0 = smem_desc_sw128(sbase + C::OFF_Q + s * C::Q_BYTES, 16, 1024);
           const uint64_t bd0 = smem_desc_sw128(kaddr, 16, 1024);
           const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
-#pragma unroll 1
+#pragma unroll
           for (int k = 0; k < D / C::UK; ++k) {
             const int c = (k * C::UK) / C::KCH;
             const int koff = ((k * C::UK) % C::KCH) * C::ELT;
-            umma_ss<C::KIND>(dcol, ad0 + static_cast<uint64_t>((c * (128 * 128) + koff) >> 4),
-                             bd0 + static_cast<uint64_t>((c * (BN * 128) + koff) >> 4), C::IDESC_S, k > 0 ? 1u : 0u);
+            umma_ss_warp<C::KIND>(dcol, ad0 + static_cast<uint64_t>((c * (128 * 128) + koff) >> 4),
+                                  bd0 + static_cast<uint64_t>((c * (BN * 128) + koff) >> 4), C::IDESC_S,
+                                  k > 0 ? 1u : 0u);
           }
-          umma_commit(&s_full[s]);
+          umma_commit_warp(&s_full[s]);
         };
         auto issue_pv = [&](int s, uint32_t vaddr, int jt) {
           const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
@@ -334,24 +340,24 @@ __global__ void __launch_bounds__(384, 1)
           // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with 4-row atoms
           // (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
           const uint64_t vd0 = DT == 0 ? smem_desc(vaddr, BN * 128, 512, 1u) : smem_desc_sw128(vaddr, BN * 128, 1024);
-#pragma unroll 1
+#pragma unroll
           for (int k = 0; k < BN / C::UK; ++k) {
             const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::UK * 128) >> 4);
             if constexpr (DT == 2) {
-              umma_ts<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-              umma_ts<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
+              umma_ts_warp<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+              umma_ts_warp<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
             } else {
-              umma_ts<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+              umma_ts_warp<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
             }
           }
-          umma_commit(&o_done[s]);
+          umma_commit_warp(&o_done[s]);
         };
         int p = 0;
         int vslot_prev = 0;
         uint32_t vaddr_prev = 0;
         for (int jt = 0; jt < n_local && ok; ++jt) {  // jt: tile index within this split
           const int kslot = p % C::NSLOT;
-          if (!mbar_wait(&kv_full[kslot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
+          if (!wait_all(&kv_full[kslot], (p / C::NSLOT) & 1)) break;
           ++p;
           tc_fence_after();
           const uint32_t kaddr = sbase + C::OFF_KV + kslot * C::KV_BYTES;
@@ -362,37 +368,38 @@ __global__ void __launch_bounds__(384, 1)
           issue_qk(0, kaddr);
           if (a.NT == 2) {
             if (jt > 0) {
-              if (!mbar_wait(&p_full[1], (jt - 1) & 1, abort_flag, a.status)) break;
+              if (!wait_all(&p_full[1], (jt - 1) & 1)) break;
               tc_fence_after();
               issue_pv(1, vaddr_prev, jt - 1);
-              umma_commit(&kv_empty[vslot_prev]);
+              umma_commit_warp(&kv_empty[vslot_prev]);
             }
             issue_qk(1, kaddr);
           }
-          umma_commit(&kv_empty[kslot]);
+          umma_commit_warp(&kv_empty[kslot]);
           const int vslot = p % C::NSLOT;
-          if (!mbar_wait(&kv_full[vslot], (p / C::NSLOT) & 1, abort_flag, a.status)) break;
+          if (!wait_all(&kv_full[vslot], (p / C::NSLOT) & 1)) break;
           ++p;
           tc_fence_after();
           const uint32_t vaddr = sbase + C::OFF_KV + vslot * C::KV_BYTES;
-          if (!mbar_wait(&p_full[0], jt & 1, abort_flag, a.status)) break;
+          if (!wait_all(&p_full[0], jt & 1)) break;
           tc_fence_after();
           issue_pv(0, vaddr, jt);
           if (a.NT == 2) {
             vslot_prev = vslot;
             vaddr_prev = vaddr;
           } else {
-            umma_commit(&kv_empty[vslot]);
+            umma_commit_warp(&kv_empty[vslot]);
           }
           if (jt == n_local - 1 && a.NT == 2) {
-            if (!mbar_wait(&p_full[1], jt & 1, abort_flag, a.status)) break;
+            if (!wait_all(&p_full[1], jt & 1)) break;
             tc_fence_after();
             issue_pv(1, vaddr, jt);
-            umma_commit(&kv_empty[vslot]);
+            umma_commit_warp(&kv_empty[vslot]);
           }
         }
-        umma_commit(mma_done);
-        mbar_wait_drain(mma_done, 0, a.status);
+        umma_commit_warp(mma_done);
+        if (lane == 0) mbar_wait_drain(mma_done, 0, a.status);
+        __syncwarp();
       }
     }
   } else {

@@ -220,6 +220,51 @@ FP2_DEVICE void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Warp-collective forms: all 32 lanes of a converged warp call them with the same (warp-uniform)
+// operands and lane 0 alone issues (predicate from %laneid inside the statement).  Keeping the
+// issuing loop warp-uniform lets descriptors and addresses stay in uniform registers, so
+// back-to-back MMAs issue without per-instruction register-to-uniform moves.  Lane 0 issues
+// every MMA and every commit, so a commit tracks all of the warp's MMAs.
+#define FP2_LANE0_PRED "{\n\t.reg .pred e, p;\n\t.reg .u32 l;\n\tmov.u32 l, %%laneid;\n\tsetp.eq.u32 e, l, 0;\n\t"
+#define FP2_UMMA_WARP_SS(KINDSTR)                                                                  \
+  asm volatile(FP2_LANE0_PRED "setp.ne.b32 p, %4, 0;\n\t"                                          \
+               "@e tcgen05.mma.cta_group::1.kind::" KINDSTR " [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem), \
+               "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)                                      \
+               : "memory")
+#define FP2_UMMA_WARP_TS(KINDSTR)                                                                  \
+  asm volatile(FP2_LANE0_PRED "setp.ne.b32 p, %4, 0;\n\t"                                          \
+               "@e tcgen05.mma.cta_group::1.kind::" KINDSTR " [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem), \
+               "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)                                     \
+               : "memory")
+
+template <int KIND>
+FP2_DEVICE void umma_ss_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
+  if constexpr (KIND == 0)
+    FP2_UMMA_WARP_SS("tf32");
+  else if constexpr (KIND == 1)
+    FP2_UMMA_WARP_SS("f16");
+  else
+    FP2_UMMA_WARP_SS("f8f6f4");
+}
+template <int KIND>
+FP2_DEVICE void umma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accum) {
+  if constexpr (KIND == 0)
+    FP2_UMMA_WARP_TS("tf32");
+  else if constexpr (KIND == 1)
+    FP2_UMMA_WARP_TS("f16");
+  else
+    FP2_UMMA_WARP_TS("f8f6f4");
+}
+FP2_DEVICE void umma_commit_warp(uint64_t* bar) {
+  asm volatile(FP2_LANE0_PRED
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+#undef FP2_UMMA_WARP_SS
+#undef FP2_UMMA_WARP_TS
+#undef FP2_LANE0_PRED
+
 // 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets row (lane base + t).
 FP2_DEVICE void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
