@@ -18,16 +18,22 @@
 // normalised partial O and its LSE, merged afterwards by combine_kernel.
 //
 // Warp roles (384 threads = 3 warpgroups):
-//   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S,
-//                    mask, online max with lazy O rescale (only when the running max grows
-//                    past a threshold), write P (bf16, f32, or e4m3 as a hi + lo pair of
-//                    planes) back over S in TMEM, and finally normalise O and store it.
+//   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S (and
+//                    release the S buffer at once), mask, online max with lazy O rescale
+//                    (only when the running max grows past a threshold), write P (bf16, f32,
+//                    or e4m3 as a hi + lo pair of planes) to the tile's P columns in TMEM, and
+//                    finally normalise O and store it.
 //   warp 8           producer: builds the kept-block bitmask, issues TMA loads of Q once and
 //                    of K/V (or kbar/vbar) tiles into an NSLOT ring of shared-memory slots.
 //   warp 9           MMA issuer (one thread): S_s = Q_s K^T (SS form) and O_s += P_s V (A
 //                    operand P read from TMEM), tcgen05.commit to mbarriers.
 //   warps 10-11      idle (they complete warpgroup 2 for the register split).
-// TMEM: S0 | S1 | O0 | O1 (512 columns); P_s aliases S_s.
+// TMEM: S | P0 | P1 | O0 | O1.  One S buffer serves both M tiles in turn: a softmax warpgroup
+// copies its S tile into registers and releases the buffer before doing any arithmetic, so
+// the next QK product (the other tile's, or this tile's next key tile) is computed while the
+// softmax runs, and the tensor pipe never waits for a whole softmax between two products of
+// the same tile.  P_s gets its own columns; the softmax writes P_s(j) only after PV_s(j-1)
+// has read P_s(j-1).
 #include <math_constants.h>
 
 #include "fp2_device.cuh"
@@ -36,7 +42,7 @@
 namespace fp2 {
 
 #ifndef REG_LOW_T
-#define REG_LOW_T 80
+#define REG_LOW_T 64
 #endif
 
 template <int DT, int D, int BN>
@@ -53,8 +59,12 @@ struct AttnCfg {
   static constexpr int TILE_BUDGET = 200 * 1024;
   static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES) / KV_BYTES;
   static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
-  static constexpr int S_COL0 = 0, S_COL1 = BN;
-  static constexpr int O_COL0 = 2 * BN, O_COL1 = 2 * BN + D;
+  // P columns per M tile: one 32-bit column per key for f32, two keys per column for bf16,
+  // two e4m3 planes of four keys per column for e4m3.
+  static constexpr int PC = DT == 0 ? BN : BN / 2;
+  static constexpr int S_COL = 0;
+  static constexpr int P_COL0 = BN, P_COL1 = BN + PC;
+  static constexpr int O_COL0 = BN + 2 * PC, O_COL1 = BN + 2 * PC + D;
   static constexpr int TMEM_COLS = 512;
   static constexpr int REG_LOW = REG_LOW_T;
   static constexpr int REG_HIGH = ((384 * 168 - 128 * REG_LOW) / 256) / 8 * 8 > 248
@@ -71,14 +81,15 @@ struct AttnCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int OFF_MASK = OFF_MISC + 16;
   // At least 116 KB so that a second CTA never shares the SM (each CTA holds all 512 TMEM columns).
-  static constexpr int SMEM_RAW = OFF_MASK + FP2_MAX_BLOCKS / 8 + 1024;
+  static constexpr int OFF_VBIAS = OFF_MASK + FP2_MAX_BLOCKS / 8;  // [2 tiles][2][BN] f32 column biases
+  static constexpr int SMEM_RAW = OFF_VBIAS + 4 * BN * 4 + 1024;
   static constexpr int SMEM_BYTES = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
-  static_assert(NSLOT >= 2, "K/V ring needs at least two slots");
-  static_assert(2 * BN + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(NSLOT >= 4, "K/V ring needs at least four slots (two key tiles in flight)");
+  static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
   static_assert(D % KCH == 0 && BN % UK == 0 && D % 32 == 0 && BN % 32 == 0, "tile shape");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -163,9 +174,11 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_done = p_full + 2;
   uint64_t* mask_ready = o_done + 2;
   uint64_t* mma_done = mask_ready + 1;
+  uint64_t* s_free = mma_done + 1;  // [2]: the S buffer has been copied out by softmax s
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
+  float* vbias = reinterpret_cast<float*>(smem + C::OFF_VBIAS);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int r, i, sub;
@@ -200,6 +213,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
       mbar_init(&o_done[s], 1);
+      mbar_init(&s_free[s], 128);
     }
     for (int k = 0; k < C::NSLOT; ++k) {
       mbar_init(&kv_full[k], 1);
@@ -259,10 +273,29 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(mask_ready);
+        // Kept blocks are taken in ascending order from the bit mask in shared memory (the same
+        // sequence as the validated column list), so the loop below makes no global reads for
+        // them.  A split starts after the kept blocks of the earlier splits.
+        const int nwords = (I >> 5) + 1;
+        int wi = 0;
+        uint32_t bits = kmask[0];
+        int skip = max(t_begin - n_virt, 0);
+        while (wi + 1 < nwords && skip >= __popc(bits)) {
+          skip -= __popc(bits);
+          bits = kmask[++wi];
+        }
+        for (; skip > 0 && bits; --skip) bits &= bits - 1;
+        auto next_kept = [&]() -> int {
+          while (bits == 0 && wi + 1 < nwords) bits = kmask[++wi];
+          if (bits == 0) return I;  // only after a rejected index (status already set)
+          const int j = (wi << 5) + __ffs(bits) - 1;
+          bits &= bits - 1;
+          return j;
+        };
         int p = 0;
         for (int jt = t_begin; jt < t_end && !*abort_flag; ++jt) {
           int j = -1;
-          if (jt >= n_virt) j = min(max(a.col_idx[rs + jt - n_virt], 0), I);
+          if (jt >= n_virt) j = next_kept();
           bool stop = false;
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
@@ -306,9 +339,11 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else if (warp == 9) {
       // ---------------------------------------------------------------- MMA issuer
-      // Ping-pong order per key tile j: QK0(j), PV1(j-1), QK1(j), PV0(j).  The softmax of tile 0
-      // then runs while the tensor pipe does PV1(j-1) and QK1(j), and the softmax of tile 1 while
-      // it does PV0(j) and QK0(j+1), so the two softmax warpgroups alternate instead of competing.
+      // Order for key tile j (NT = 2): QK1(j), PV1(j-1), QK0(j+1), PV0(j).  QK products only
+      // wait for the S buffer (the previous softmax has copied its S tile out) and their K tile;
+      // PV_s(j) waits for P_s(j).  Softmax 0 works on tile j while the pipe runs QK1(j),
+      // PV1(j-1) and QK0(j+1), so S0(j+1) is ready when it finishes, and symmetrically for
+      // softmax 1.  With NT = 1: QK0(j+1), PV0(j).
       // The whole warp runs this loop with warp-uniform control flow (every wait is voted) and
       // lane 0 issues each tcgen05 instruction (the *_warp wrappers).
       {
@@ -323,8 +358,8 @@ __global__ void __launch_bounds__(384, 1)
         auto issue_qk = [&](int s, uint32_t kaddr) {
           const uint64_t ad0 = smem_desc_sw128(sbase + C::OFF_Q + s * C::Q_BYTES, 16, 1024);
           const uint64_t bd0 = smem_desc_sw128(kaddr, 16, 1024);
-          const uint32_t dcol = tmem + (s ? C::S_COL1 : C::S_COL0);
-#pragma unroll
+          const uint32_t dcol = tmem + C::S_COL;
+#pragma unroll 1
           for (int k = 0; k < D / C::UK; ++k) {
             const int c = (k * C::UK) / C::KCH;
             const int koff = ((k * C::UK) % C::KCH) * C::ELT;
@@ -335,12 +370,12 @@ __global__ void __launch_bounds__(384, 1)
           umma_commit_warp(&s_full[s]);
         };
         auto issue_pv = [&](int s, uint32_t vaddr, int jt) {
-          const uint32_t pcol = tmem + (s ? C::S_COL1 : C::S_COL0);
+          const uint32_t pcol = tmem + (s ? C::P_COL1 : C::P_COL0);
           const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
           // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with 4-row atoms
           // (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
           const uint64_t vd0 = DT == 0 ? smem_desc(vaddr, BN * 128, 512, 1u) : smem_desc_sw128(vaddr, BN * 128, 1024);
-#pragma unroll
+#pragma unroll 1
           for (int k = 0; k < BN / C::UK; ++k) {
             const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::UK * 128) >> 4);
             if constexpr (DT == 2) {
@@ -352,49 +387,49 @@ __global__ void __launch_bounds__(384, 1)
           }
           umma_commit_warp(&o_done[s]);
         };
-        int p = 0;
-        int vslot_prev = 0;
-        uint32_t vaddr_prev = 0;
+        // Loads come in the order K(0), V(0), K(1), V(1), ...: K(j) is load 2j, V(j) load 2j+1.
+        auto slot_of = [&](int q) { return q % C::NSLOT; };
+        auto kv_wait = [&](int q) { return wait_all(&kv_full[slot_of(q)], (q / C::NSLOT) & 1); };
+        auto slot_addr = [&](int q) { return sbase + C::OFF_KV + slot_of(q) * C::KV_BYTES; };
+        if (n_local > 0 && ok) {
+          ok = kv_wait(0);
+          if (ok) {
+            tc_fence_after();
+            issue_qk(0, slot_addr(0));
+            if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(0)]);
+          }
+        }
         for (int jt = 0; jt < n_local && ok; ++jt) {  // jt: tile index within this split
-          const int kslot = p % C::NSLOT;
-          if (!wait_all(&kv_full[kslot], (p / C::NSLOT) & 1)) break;
-          ++p;
-          tc_fence_after();
-          const uint32_t kaddr = sbase + C::OFF_KV + kslot * C::KV_BYTES;
-          // QK_s(j) is issued right behind PV_s(j-1) without waiting for it: the tensor pipe runs
-          // one thread's MMAs in issue order, so PV_s(j-1) has read P_s out of the S_s columns
-          // before QK_s(j) overwrites them, and s_full (a commit) also covers PV_s(j-1), so the
-          // softmax never sees O_s mid-update.
-          issue_qk(0, kaddr);
+          const int qk = 2 * jt, qv = 2 * jt + 1;
           if (a.NT == 2) {
+            if (!wait_all(&s_free[0], jt & 1)) break;  // softmax 0 holds S0(jt)
+            tc_fence_after();
+            issue_qk(1, slot_addr(qk));
+            umma_commit_warp(&kv_empty[slot_of(qk)]);  // K(jt) fully consumed
             if (jt > 0) {
               if (!wait_all(&p_full[1], (jt - 1) & 1)) break;
               tc_fence_after();
-              issue_pv(1, vaddr_prev, jt - 1);
-              umma_commit_warp(&kv_empty[vslot_prev]);
+              issue_pv(1, slot_addr(qv - 2), jt - 1);
+              umma_commit_warp(&kv_empty[slot_of(qv - 2)]);  // V(jt-1) fully consumed
             }
-            issue_qk(1, kaddr);
           }
-          umma_commit_warp(&kv_empty[kslot]);
-          const int vslot = p % C::NSLOT;
-          if (!wait_all(&kv_full[vslot], (p / C::NSLOT) & 1)) break;
-          ++p;
-          tc_fence_after();
-          const uint32_t vaddr = sbase + C::OFF_KV + vslot * C::KV_BYTES;
+          if (jt + 1 < n_local) {
+            if (!kv_wait(qk + 2)) break;
+            if (!wait_all(&s_free[a.NT - 1], jt & 1)) break;  // the last softmax holds its S(jt)
+            tc_fence_after();
+            issue_qk(0, slot_addr(qk + 2));
+            if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(qk + 2)]);
+          }
+          if (!kv_wait(qv)) break;
           if (!wait_all(&p_full[0], jt & 1)) break;
           tc_fence_after();
-          issue_pv(0, vaddr, jt);
-          if (a.NT == 2) {
-            vslot_prev = vslot;
-            vaddr_prev = vaddr;
-          } else {
-            umma_commit_warp(&kv_empty[vslot]);
-          }
-          if (jt == n_local - 1 && a.NT == 2) {
+          issue_pv(0, slot_addr(qv), jt);
+          if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(qv)]);
+          if (a.NT == 2 && jt == n_local - 1) {
             if (!wait_all(&p_full[1], jt & 1)) break;
             tc_fence_after();
-            issue_pv(1, vaddr, jt);
-            umma_commit_warp(&kv_empty[vslot]);
+            issue_pv(1, slot_addr(qv), jt);
+            umma_commit_warp(&kv_empty[slot_of(qv)]);
           }
         }
         umma_commit_warp(mma_done);
@@ -414,7 +449,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool row_ok = (hl < a.G) && (i * BN + tl < L);
       const int h = g * a.G + min(hl, a.G - 1);
       const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-      const uint32_t s_addr = tmem + lane_base + (s ? C::S_COL1 : C::S_COL0);
+      const uint32_t s_addr = tmem + lane_base + C::S_COL;
+      const uint32_t p_addr = tmem + lane_base + (s ? C::P_COL1 : C::P_COL0);
       const uint32_t o_addr = tmem + lane_base + (s ? C::O_COL1 : C::O_COL0);
       const float s2 = a.sm_scale_log2;
       const float bias_raw = a.log2_blk / s2;
@@ -432,17 +468,48 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld128_sync(s_addr, v);
         else
           tmem_ld64_sync(s_addr, v);
+        // S is in registers: hand the buffer to the next QK product.
+        tc_fence_before();
+        mbar_arrive(&s_free[s]);
+        // PV_s(jl-1) must be complete before O_s is rescaled or P_s is overwritten.
+        bool pv_prev_done = jl == 0;
+        auto wait_pv_prev = [&]() {
+          if (!pv_prev_done) {
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (jl - 1) & 1, abort_flag, a.status));
+            tc_fence_after();
+            pv_prev_done = true;
+          }
+          return ok;
+        };
         // Tile kinds: virtual (pooled keys of blocks [jt*BN, jt*BN+BN): only pruned blocks, with the
         // ln n_j bias), diagonal (causal mask), full (no mask).  The mask works on raw S values:
         // x = S * s2 with s2 > 0, so the bias is added as log2(n)/s2 and the max is taken on raw S.
         float xs[BN];
         if (jt < n_virt) {
+          // The column mask and bias of a virtual tile are the same for every row of the CTA, so
+          // the warpgroup builds them once as a row of f32 biases in shared memory (thread t:
+          // pooled block jt*BN + t; +log2(n)/s2 for a pruned block, -inf otherwise) and every
+          // row adds that row.  Two buffers alternate by tile: a thread writes the buffer of
+          // tile jt + 2 only after the barrier of tile jt + 1, which every thread reaches after
+          // its reads of tile jt (virtual tiles are consecutive, and each has the barrier).
+          float* vb = vbias + (2 * s + (jt & 1)) * BN;
+          if (rt < BN) {
+            const int blk = jt * BN + rt;
+            const bool pr = blk < I && !((kmask[blk >> 5] >> (blk & 31)) & 1u);
+            vb[rt] = pr ? bias_raw : -CUDART_INF_F;
+          }
+          asm volatile("bar.sync %0, 128;" ::"r"(1 + s) : "memory");
   #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            const uint32_t word = pruned_word(kmask, jt * BN + c * 32, I);
-  #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              xs[c * 32 + e] = ((word >> e) & 1u) ? __uint_as_float(v[c * 32 + e]) + bias_raw : -CUDART_INF_F;
+          for (int e = 0; e < BN; e += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(vb + e);
+            const float2 x01 = __fadd2_rn(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
+                                          make_float2(b4.x, b4.y));
+            const float2 x23 = __fadd2_rn(make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
+                                          make_float2(b4.z, b4.w));
+            xs[e] = x01.x;
+            xs[e + 1] = x01.y;
+            xs[e + 2] = x23.x;
+            xs[e + 3] = x23.y;
           }
         } else if (jt == n_tiles - 1) {
   #pragma unroll
@@ -464,6 +531,7 @@ __global__ void __launch_bounds__(384, 1)
         const float m_new = fmaxf(m_run, mt);
         const bool need = m_new > m_run + C::LAZY;
         if (jl > 0 && __any_sync(0xFFFFFFFFu, need)) {
+          if (!wait_pv_prev()) break;
           const float f = need ? fast_exp2(m_run - m_new) : 1.0f;
   #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -484,7 +552,7 @@ __global__ void __launch_bounds__(384, 1)
           l_run = (m_run == -CUDART_INF_F) ? 0.f : l_run * fast_exp2(m_run - m_new);
           m_run = m_new;
         }
-        // P = 2^(S*s2 - m + P_SHIFT), packed to the MMA operand type and written over S in TMEM.
+        // P = 2^(S*s2 - m + P_SHIFT), packed to the MMA operand type and written to P_s in TMEM.
         const float nmu = C::P_SHIFT - ((m_run == -CUDART_INF_F) ? 0.f : m_run);
         // Exponent arguments x * s2 + nmu and the row sums in packed f32x2 arithmetic (pairs of
         // adjacent scores); the same fused multiply-add as the scalar form, so P is unchanged.
@@ -497,27 +565,36 @@ __global__ void __launch_bounds__(384, 1)
           return p;
         };
         if constexpr (DT == 1) {
-          uint32_t pk[BN / 2];
+          // 64 scores -> 32 packed words -> one TMEM store, chunk by chunk (keeps fewer P words live).
   #pragma unroll
-          for (int e = 0; e < BN / 2; ++e) {
-            const float2 p = exp_pair(e);
-            pk[e] = pack_bf16x2(p.x, p.y);
-          }
+          for (int c = 0; c < BN / 64; ++c) {
+            uint32_t pk[32];
   #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
-        } else if constexpr (DT == 2) {
-          // K-step c (32 keys) of the PV MMA: hi plane at columns [16c, 16c+8), lo at [16c+8, 16c+16).
-          uint32_t pk[BN / 2];
-  #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-  #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float2 pa = exp_pair(c * 16 + 2 * e), pb = exp_pair(c * 16 + 2 * e + 1);
-              split_e4m3x4(pa.x, pa.y, pb.x, pb.y, pk[c * 16 + e], pk[c * 16 + 8 + e]);
+            for (int e = 0; e < 32; ++e) {
+              const float2 p = exp_pair(c * 32 + e);
+              pk[e] = pack_bf16x2(p.x, p.y);
             }
+            if (c == 0 && !wait_pv_prev()) break;
+            tmem_st32(p_addr + c * 32, pk);
           }
+        } else if constexpr (DT == 2) {
+          // K-step c (32 keys) of the PV MMA: hi plane at columns [16c, 16c+8), lo at [16c+8, 16c+16);
+          // two K-steps (32 words) per TMEM store.
   #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
+          for (int h = 0; h < BN / 64; ++h) {
+            uint32_t pk[32];
+  #pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int c = 2 * h + cc;
+                const float2 pa = exp_pair(c * 16 + 2 * e), pb = exp_pair(c * 16 + 2 * e + 1);
+                split_e4m3x4(pa.x, pa.y, pb.x, pb.y, pk[cc * 16 + e], pk[cc * 16 + 8 + e]);
+              }
+            }
+            if (h == 0 && !wait_pv_prev()) break;
+            tmem_st32(p_addr + h * 32, pk);
+          }
         } else {
           uint32_t pk[BN];
   #pragma unroll
@@ -526,9 +603,12 @@ __global__ void __launch_bounds__(384, 1)
             pk[2 * e] = __float_as_uint(p.x);
             pk[2 * e + 1] = __float_as_uint(p.y);
           }
+          if (wait_pv_prev()) {
   #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) tmem_st32(s_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
+            for (int c = 0; c < BN / 32; ++c) tmem_st32(p_addr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&pk[c * 32]));
+          }
         }
+        if (!ok) break;
         const float rsum = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
         tmem_st_wait();
         tc_fence_before();

@@ -103,7 +103,22 @@ FP2_DEVICE void setmaxnreg_dec() {
 // waits without a limit.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
+// Non-blocking probe of the phase (no suspend): the cheap first check of a wait that is often
+// already satisfied.
+FP2_DEVICE bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 FP2_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
+  if (mbar_test_wait(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
