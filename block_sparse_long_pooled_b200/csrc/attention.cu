@@ -25,9 +25,13 @@
 //                    finally normalise O and store it.
 //   warp 8           producer: builds the kept-block bitmask, issues TMA loads of Q once and
 //                    of K/V (or kbar/vbar) tiles into an NSLOT ring of shared-memory slots.
-//   warp 9           MMA issuer (one thread): S_s = Q_s K^T (SS form) and O_s += P_s V (A
-//                    operand P read from TMEM), tcgen05.commit to mbarriers.
-//   warps 10-11      idle (they complete warpgroup 2 for the register split).
+//   warp 9           QK issuer: S = Q_s K^T (SS form) into the shared S buffer.
+//   warp 10          PV issuer: O_s += P_s V (A operand P_s read from TMEM).  The two products
+//                    touch disjoint TMEM, so each is issued the moment its own inputs are ready
+//                    and the tensor pipe interleaves them; one issuer would stall the pipe at
+//                    every wait between groups.  Both issue tcgen05.mma from lane 0 and signal
+//                    mbarriers with tcgen05.commit.
+//   warp 11          idle (it completes warpgroup 2 for the register split).
 // TMEM: S | P0 | P1 | O0 | O1.  One S buffer serves both M tiles in turn: a softmax warpgroup
 // copies its S tile into registers and releases the buffer before doing any arithmetic, so
 // the next QK product (the other tile's, or this tile's next key tile) is computed while the
@@ -81,8 +85,8 @@ struct AttnCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int OFF_MISC = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
   static constexpr int OFF_MASK = OFF_MISC + 16;
   // At least 116 KB so that a second CTA never shares the SM (each CTA holds all 512 TMEM columns).
   static constexpr int OFF_VBIAS = OFF_MASK + FP2_MAX_BLOCKS / 8;  // [2 tiles][2][BN] f32 column biases
@@ -90,6 +94,7 @@ struct AttnCfg {
   static constexpr int SMEM_BYTES = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
   static_assert(NSLOT >= 4, "K/V ring needs at least four slots (two key tiles in flight)");
   static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
+  static_assert(OFF_BAR % 8 == 0 && OFF_MASK % 16 == 0 && OFF_VBIAS % 16 == 0, "shared-memory alignment");
   static_assert(D % KCH == 0 && BN % UK == 0 && D % 32 == 0 && BN % 32 == 0, "tile shape");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -175,6 +180,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* mask_ready = o_done + 2;
   uint64_t* mma_done = mask_ready + 1;
   uint64_t* s_free = mma_done + 1;  // [2]: the S buffer has been copied out by softmax s
+  uint64_t* pv_done = s_free + 2;   // the PV issuer's final commit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
@@ -221,6 +227,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(mask_ready, 1);
     mbar_init(mma_done, 1);
+    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -337,104 +344,102 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status);
         for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status);
       }
-    } else if (warp == 9) {
-      // ---------------------------------------------------------------- MMA issuer
-      // Order for key tile j (NT = 2): QK1(j), PV1(j-1), QK0(j+1), PV0(j).  QK products only
-      // wait for the S buffer (the previous softmax has copied its S tile out) and their K tile;
-      // PV_s(j) waits for P_s(j).  Softmax 0 works on tile j while the pipe runs QK1(j),
-      // PV1(j-1) and QK0(j+1), so S0(j+1) is ready when it finishes, and symmetrically for
-      // softmax 1.  With NT = 1: QK0(j+1), PV0(j).
-      // The whole warp runs this loop with warp-uniform control flow (every wait is voted) and
-      // lane 0 issues each tcgen05 instruction (the *_warp wrappers).
+    } else if (warp == 9 || warp == 10) {
+      // ---------------------------------------------------------------- MMA issuers
+      // QK issuer (warp 9), for key tile j with NT = 2: QK1(j) once softmax 0 has copied S0(j)
+      // out, then QK0(j+1) once softmax 1 has copied S1(j) out; NT = 1: QK0(j+1) after S0(j).
+      // PV issuer (warp 10): PV0(j) once P0(j) is written, then PV1(j).
+      // Each warp runs its loop with warp-uniform control flow (every wait is voted) and lane 0
+      // issues each tcgen05 instruction (the *_warp wrappers).
       {
         auto wait_all = [&](uint64_t* bar, uint32_t parity) {
           return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, a.status));
-        };
-        bool ok = true;
-        for (int s = 0; s < a.NT && ok; ++s) ok = wait_all(&q_full[s], 0);
-        tc_fence_after();
-        // Descriptors are formed once per tile; a K step only moves the start address, which is
-        // the low 14 bits (address >> 4) of the descriptor and cannot carry (shared memory < 256 KB).
-        auto issue_qk = [&](int s, uint32_t kaddr) {
-          const uint64_t ad0 = smem_desc_sw128(sbase + C::OFF_Q + s * C::Q_BYTES, 16, 1024);
-          const uint64_t bd0 = smem_desc_sw128(kaddr, 16, 1024);
-          const uint32_t dcol = tmem + C::S_COL;
-#pragma unroll 1
-          for (int k = 0; k < D / C::UK; ++k) {
-            const int c = (k * C::UK) / C::KCH;
-            const int koff = ((k * C::UK) % C::KCH) * C::ELT;
-            umma_ss_warp<C::KIND>(dcol, ad0 + static_cast<uint64_t>((c * (128 * 128) + koff) >> 4),
-                                  bd0 + static_cast<uint64_t>((c * (BN * 128) + koff) >> 4), C::IDESC_S,
-                                  k > 0 ? 1u : 0u);
-          }
-          umma_commit_warp(&s_full[s]);
-        };
-        auto issue_pv = [&](int s, uint32_t vaddr, int jt) {
-          const uint32_t pcol = tmem + (s ? C::P_COL1 : C::P_COL0);
-          const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
-          // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with 4-row atoms
-          // (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
-          const uint64_t vd0 = DT == 0 ? smem_desc(vaddr, BN * 128, 512, 1u) : smem_desc_sw128(vaddr, BN * 128, 1024);
-#pragma unroll 1
-          for (int k = 0; k < BN / C::UK; ++k) {
-            const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::UK * 128) >> 4);
-            if constexpr (DT == 2) {
-              umma_ts_warp<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-              umma_ts_warp<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
-            } else {
-              umma_ts_warp<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-            }
-          }
-          umma_commit_warp(&o_done[s]);
         };
         // Loads come in the order K(0), V(0), K(1), V(1), ...: K(j) is load 2j, V(j) load 2j+1.
         auto slot_of = [&](int q) { return q % C::NSLOT; };
         auto kv_wait = [&](int q) { return wait_all(&kv_full[slot_of(q)], (q / C::NSLOT) & 1); };
         auto slot_addr = [&](int q) { return sbase + C::OFF_KV + slot_of(q) * C::KV_BYTES; };
-        if (n_local > 0 && ok) {
-          ok = kv_wait(0);
-          if (ok) {
-            tc_fence_after();
-            issue_qk(0, slot_addr(0));
-            if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(0)]);
-          }
-        }
-        for (int jt = 0; jt < n_local && ok; ++jt) {  // jt: tile index within this split
-          const int qk = 2 * jt, qv = 2 * jt + 1;
-          if (a.NT == 2) {
-            if (!wait_all(&s_free[0], jt & 1)) break;  // softmax 0 holds S0(jt)
-            tc_fence_after();
-            issue_qk(1, slot_addr(qk));
-            umma_commit_warp(&kv_empty[slot_of(qk)]);  // K(jt) fully consumed
-            if (jt > 0) {
-              if (!wait_all(&p_full[1], (jt - 1) & 1)) break;
+        bool ok = true;
+        if (warp == 9) {
+          for (int s = 0; s < a.NT && ok; ++s) ok = wait_all(&q_full[s], 0);
+          tc_fence_after();
+          // Descriptors are formed once per tile; a K step only moves the start address, which is
+          // the low 14 bits (address >> 4) of the descriptor and cannot carry (smem < 256 KB).
+          auto issue_qk = [&](int s, uint32_t kaddr) {
+            const uint64_t ad0 = smem_desc_sw128(sbase + C::OFF_Q + s * C::Q_BYTES, 16, 1024);
+            const uint64_t bd0 = smem_desc_sw128(kaddr, 16, 1024);
+            const uint32_t dcol = tmem + C::S_COL;
+#pragma unroll 1
+            for (int k = 0; k < D / C::UK; ++k) {
+              const int c = (k * C::UK) / C::KCH;
+              const int koff = ((k * C::UK) % C::KCH) * C::ELT;
+              umma_ss_warp<C::KIND>(dcol, ad0 + static_cast<uint64_t>((c * (128 * 128) + koff) >> 4),
+                                    bd0 + static_cast<uint64_t>((c * (BN * 128) + koff) >> 4), C::IDESC_S,
+                                    k > 0 ? 1u : 0u);
+            }
+            umma_commit_warp(&s_full[s]);
+          };
+          if (n_local > 0 && ok) {
+            ok = kv_wait(0);
+            if (ok) {
               tc_fence_after();
-              issue_pv(1, slot_addr(qv - 2), jt - 1);
-              umma_commit_warp(&kv_empty[slot_of(qv - 2)]);  // V(jt-1) fully consumed
+              issue_qk(0, slot_addr(0));
+              if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(0)]);
             }
           }
-          if (jt + 1 < n_local) {
-            if (!kv_wait(qk + 2)) break;
-            if (!wait_all(&s_free[a.NT - 1], jt & 1)) break;  // the last softmax holds its S(jt)
-            tc_fence_after();
-            issue_qk(0, slot_addr(qk + 2));
-            if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(qk + 2)]);
+          for (int jt = 0; jt < n_local && ok; ++jt) {  // jt: tile index within this split
+            const int qk = 2 * jt;
+            if (a.NT == 2) {
+              if (!wait_all(&s_free[0], jt & 1)) break;  // softmax 0 holds S0(jt)
+              tc_fence_after();
+              issue_qk(1, slot_addr(qk));
+              umma_commit_warp(&kv_empty[slot_of(qk)]);  // K(jt) fully consumed
+            }
+            if (jt + 1 < n_local) {
+              if (!kv_wait(qk + 2)) break;
+              if (!wait_all(&s_free[a.NT - 1], jt & 1)) break;  // the last softmax holds its S(jt)
+              tc_fence_after();
+              issue_qk(0, slot_addr(qk + 2));
+              if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(qk + 2)]);
+            }
           }
-          if (!kv_wait(qv)) break;
-          if (!wait_all(&p_full[0], jt & 1)) break;
-          tc_fence_after();
-          issue_pv(0, slot_addr(qv), jt);
-          if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(qv)]);
-          if (a.NT == 2 && jt == n_local - 1) {
-            if (!wait_all(&p_full[1], jt & 1)) break;
-            tc_fence_after();
-            issue_pv(1, slot_addr(qv), jt);
-            umma_commit_warp(&kv_empty[slot_of(qv)]);
+          umma_commit_warp(mma_done);
+          if (lane == 0) mbar_wait_drain(mma_done, 0, a.status);
+          __syncwarp();
+        } else {
+          auto issue_pv = [&](int s, uint32_t vaddr, int jt) {
+            const uint32_t pcol = tmem + (s ? C::P_COL1 : C::P_COL0);
+            const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
+            // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with 4-row
+            // atoms (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
+            const uint64_t vd0 = DT == 0 ? smem_desc(vaddr, BN * 128, 512, 1u) : smem_desc_sw128(vaddr, BN * 128, 1024);
+#pragma unroll 1
+            for (int k = 0; k < BN / C::UK; ++k) {
+              const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::UK * 128) >> 4);
+              if constexpr (DT == 2) {
+                umma_ts_warp<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+                umma_ts_warp<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
+              } else {
+                umma_ts_warp<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
+              }
+            }
+            umma_commit_warp(&o_done[s]);
+          };
+          for (int jt = 0; jt < n_local && ok; ++jt) {
+            const int qv = 2 * jt + 1;
+            if (!kv_wait(qv)) break;
+            for (int s = 0; s < a.NT; ++s) {
+              if (!(ok = wait_all(&p_full[s], jt & 1))) break;
+              tc_fence_after();
+              issue_pv(s, slot_addr(qv), jt);
+            }
+            if (!ok) break;
+            umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
           }
+          umma_commit_warp(pv_done);
+          if (lane == 0) mbar_wait_drain(pv_done, 0, a.status);
+          __syncwarp();
         }
-        umma_commit_warp(mma_done);
-        if (lane == 0) mbar_wait_drain(mma_done, 0, a.status);
-        __syncwarp();
       }
     }
   } else {
