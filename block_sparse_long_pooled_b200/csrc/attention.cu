@@ -85,16 +85,23 @@ struct AttnCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2;
+  // Output staging for TMA stores: tile s's normalised O (128 rows x d, output type) goes into
+  // the shared memory of its own Q tile, free once the tile's last QK product is done; only when
+  // it fits there (bf16 and f32 inputs; e4m3 Q tiles are half the size of a bf16 O tile).
+  static constexpr int OUT_ELT = DT == 0 ? 4 : 2;
+  static constexpr int OCH = 128 / OUT_ELT;          // output elements per 128-byte box row
+  static constexpr int OBOX = BN * 128;              // one box: BN rows x 128 bytes
+  static constexpr int O_STAGE_BYTES = 128 * D * OUT_ELT;
+  static constexpr bool TMA_OUT = O_STAGE_BYTES <= Q_BYTES;
   static constexpr int OFF_MISC = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
   static constexpr int OFF_MASK = OFF_MISC + 16;
   // At least 116 KB so that a second CTA never shares the SM (each CTA holds all 512 TMEM columns).
-  static constexpr int OFF_VBIAS = OFF_MASK + FP2_MAX_BLOCKS / 8;  // [2 tiles][2][BN] f32 column biases
-  static constexpr int SMEM_RAW = OFF_VBIAS + 4 * BN * 4 + 1024;
+  static constexpr int SMEM_RAW = OFF_MASK + FP2_MAX_BLOCKS / 8 + 1024;
   static constexpr int SMEM_BYTES = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
   static_assert(NSLOT >= 4, "K/V ring needs at least four slots (two key tiles in flight)");
   static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
-  static_assert(OFF_BAR % 8 == 0 && OFF_MASK % 16 == 0 && OFF_VBIAS % 16 == 0, "shared-memory alignment");
+  static_assert(OFF_BAR % 8 == 0 && OFF_MASK % 16 == 0, "shared-memory alignment");
   static_assert(D % KCH == 0 && BN % UK == 0 && D % 32 == 0 && BN % 32 == 0, "tile shape");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -181,10 +188,10 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* mma_done = mask_ready + 1;
   uint64_t* s_free = mma_done + 1;  // [2]: the S buffer has been copied out by softmax s
   uint64_t* pv_done = s_free + 2;   // the PV issuer's final commit
+  uint64_t* o_staged = pv_done + 1; // [2]: every row of tile s is staged for the TMA store
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
-  float* vbias = reinterpret_cast<float*>(smem + C::OFF_VBIAS);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int r, i, sub;
@@ -220,6 +227,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&p_full[s], 128);
       mbar_init(&o_done[s], 1);
       mbar_init(&s_free[s], 128);
+      mbar_init(&o_staged[s], 128);
     }
     for (int k = 0; k < C::NSLOT; ++k) {
       mbar_init(&kv_full[k], 1);
@@ -461,6 +469,7 @@ __global__ void __launch_bounds__(384, 1)
       const float bias_raw = a.log2_blk / s2;
       float m_run = -CUDART_INF_F, l_run = 0.f;
       bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status));
+
       int done_tiles = 0;
       for (int jl = 0; jl < n_local && ok; ++jl) {
         const int jt = t_begin + jl;  // position in the row's key stream
@@ -491,30 +500,22 @@ __global__ void __launch_bounds__(384, 1)
         // x = S * s2 with s2 > 0, so the bias is added as log2(n)/s2 and the max is taken on raw S.
         float xs[BN];
         if (jt < n_virt) {
-          // The column mask and bias of a virtual tile are the same for every row of the CTA, so
-          // the warpgroup builds them once as a row of f32 biases in shared memory (thread t:
-          // pooled block jt*BN + t; +log2(n)/s2 for a pruned block, -inf otherwise) and every
-          // row adds that row.  Two buffers alternate by tile: a thread writes the buffer of
-          // tile jt + 2 only after the barrier of tile jt + 1, which every thread reaches after
-          // its reads of tile jt (virtual tiles are consecutive, and each has the barrier).
-          float* vb = vbias + (2 * s + (jt & 1)) * BN;
-          if (rt < BN) {
-            const int blk = jt * BN + rt;
-            const bool pr = blk < I && !((kmask[blk >> 5] >> (blk & 31)) & 1u);
-            vb[rt] = pr ? bias_raw : -CUDART_INF_F;
-          }
-          asm volatile("bar.sync %0, 128;" ::"r"(1 + s) : "memory");
+          // The column mask and bias of a virtual tile are the same for every row of the CTA:
+          // lane l of each warp works out the bias of columns l, l + 32, ... (+log2(n)/s2 for a
+          // pruned block, -inf otherwise) and every row gets them by warp shuffles.
   #pragma unroll
-          for (int e = 0; e < BN; e += 4) {
-            const float4 b4 = *reinterpret_cast<const float4*>(vb + e);
-            const float2 x01 = __fadd2_rn(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])),
-                                          make_float2(b4.x, b4.y));
-            const float2 x23 = __fadd2_rn(make_float2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])),
-                                          make_float2(b4.z, b4.w));
-            xs[e] = x01.x;
-            xs[e + 1] = x01.y;
-            xs[e + 2] = x23.x;
-            xs[e + 3] = x23.y;
+          for (int c = 0; c < BN / 32; ++c) {
+            const int blk = jt * BN + c * 32 + lane;
+            const bool pr = blk < I && !((kmask[blk >> 5] >> (blk & 31)) & 1u);
+            const float bias_l = pr ? bias_raw : -CUDART_INF_F;
+  #pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float2 x2 = __fadd2_rn(
+                  make_float2(__uint_as_float(v[c * 32 + e]), __uint_as_float(v[c * 32 + e + 1])),
+                  make_float2(__shfl_sync(0xFFFFFFFFu, bias_l, e), __shfl_sync(0xFFFFFFFFu, bias_l, e + 1)));
+              xs[c * 32 + e] = x2.x;
+              xs[c * 32 + e + 1] = x2.y;
+            }
           }
         } else if (jt == n_tiles - 1) {
   #pragma unroll
@@ -652,6 +653,54 @@ __global__ void __launch_bounds__(384, 1)
         if (row_ok)
           a.lse_part[(static_cast<int64_t>(split) * a.Hq + h) * a.total_tokens + tok] =
               any ? (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f : -CUDART_INF_F;
+      } else if (C::TMA_OUT && a.o_tma && i * BN + BN <= L) {
+        // Full block: every thread writes its normalised row into the tile's staging buffer in
+        // the 128-byte-swizzled box layout of tm_o (16-byte chunk c of box row t at c ^ (t & 7)),
+        // then one thread stores the boxes with TMA once all 128 rows are staged.  All threads
+        // arrive on o_staged whatever happened before, so the bounded wait below always ends.
+        uint8_t* stg = smem + C::OFF_Q + s * C::Q_BYTES;  // inside tile s's own Q buffer
+        if (ok) {
+          const float inv = a.v_descale / l_run;
+  #pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32_sync(o_addr + c * 32, v);
+  #pragma unroll
+            for (int q = 0; q < 32 * C::OUT_ELT / 16; ++q) {
+              uint4 w;
+              if constexpr (DT == 0) {
+                w = make_uint4(__float_as_uint(__uint_as_float(v[4 * q]) * inv),
+                               __float_as_uint(__uint_as_float(v[4 * q + 1]) * inv),
+                               __float_as_uint(__uint_as_float(v[4 * q + 2]) * inv),
+                               __float_as_uint(__uint_as_float(v[4 * q + 3]) * inv));
+              } else {
+                w.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv);
+              }
+              const int off = c * 32 * C::OUT_ELT + q * 16;  // byte offset of this chunk in the row
+              const int k = off / 128, ci = (off % 128) / 16;
+              *reinterpret_cast<uint4*>(stg + (k * HS + hs) * C::OBOX + tl * 128 + ((ci ^ (tl & 7)) * 16)) = w;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&o_staged[s]);
+        if (qd == 0 && lane == 0 && mbar_wait(&o_staged[s], 0, abort_flag, a.status) && !*abort_flag) {
+          const int tok0 = P.tok_off[r] + i * BN;
+          for (int hs2 = 0; hs2 < HS; ++hs2) {
+            const int hl2 = (part * a.NT + s) * HS + hs2;
+            if (hl2 >= a.G) continue;
+            for (int k = 0; k < D / C::OCH; ++k)
+              tma_store_3d(&a.tm_o, stg + (k * HS + hs2) * C::OBOX, k * C::OCH, g * a.G + hl2, tok0);
+          }
+          bulk_commit_group();
+          bulk_wait_read_all();
+        }
+        if (ok && row_ok && a.lse != nullptr)
+          a.lse[static_cast<int64_t>(h) * a.total_tokens + P.tok_off[r] + i * BN + tl] =
+              (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f;
       } else if (ok) {
         const int tok = P.tok_off[r] + i * BN + tl;
         const float inv = a.v_descale / l_run;

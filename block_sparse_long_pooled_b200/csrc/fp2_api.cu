@@ -354,6 +354,15 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
     return st2;
   if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_k_blocks, hd, B, v32)) != FP2_OK)
     return st2;
+  // Output tiles of full blocks go out through TMA stores (16-byte aligned output, no KV split);
+  // everything else through per-thread stores.
+  if (c.splits == 1 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+    const fp2_dtype odt = p->dtype == FP2_F32 ? FP2_F32 : FP2_BF16;
+    a.o_tma = encode_3d(&a.tm_o, odt, out, D, p->num_q_heads, c.T, static_cast<int64_t>(p->num_q_heads) * D, B) ==
+                      FP2_OK
+                  ? 1
+                  : 0;
+  }
   a.row_ptr = ix->row_ptr;
   a.col_idx = ix->col_idx;
   a.page_table = p->page_table;

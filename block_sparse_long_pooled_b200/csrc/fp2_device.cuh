@@ -146,6 +146,20 @@ FP2_DEVICE void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, in
       : "memory");
 }
 
+// TMA tile store from shared memory (bulk-group completion).  Coordinates are never negative and
+// the innermost one is a multiple of 16 bytes.
+FP2_DEVICE void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+FP2_DEVICE void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store has finished reading its shared-memory source.
+FP2_DEVICE void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Make this thread's generic-proxy shared-memory writes visible to the async (TMA) proxy.
+FP2_DEVICE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ------------------------------------------------------------------ tcgen05
 
 FP2_DEVICE void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

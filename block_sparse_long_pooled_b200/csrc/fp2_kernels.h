@@ -49,6 +49,8 @@ struct AttnArgs {
   CUtensorMap tm_v;
   CUtensorMap tm_kb;  // kbar_mma [blocks, Hkv, d] box {128B / elt, 1, B}
   CUtensorMap tm_vb;
+  CUtensorMap tm_o;   // out [T, Hq, d] (bf16, or f32 for f32 inputs) box {128B / elt, 1, B}
+  int o_tma;          // 1: full blocks are written through tm_o by TMA stores
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const int32_t* page_table;  // NULL -> contiguous
