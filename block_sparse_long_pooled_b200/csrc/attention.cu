@@ -251,7 +251,42 @@ __global__ void __launch_bounds__(384, 1)
     setmaxnreg_dec<C::REG_LOW>();
     if (warp == 8) {
       // ---------------------------------------------------------------- producer
-      // Q first (it has no dependency), then the kept-block mask while Q is in flight.
+      // Q and the first key tiles first (they need no mask), then the kept-block mask while
+      // they are in flight, then the remaining key tiles as ring slots free up.
+      // Load p of this CTA goes to slot p % NSLOT: K of tile t is load 2t, V load 2t+1.
+      auto issue_kv = [&](int jt, int j, int q, int kv) {
+        const int slot = q % C::NSLOT;
+        mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
+        uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
+        if (j < 0) {
+          const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_blk_off[r] + jt * BN);
+        } else if (a.page_table == nullptr) {
+          const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
+          for (int c = 0; c < C::DCH; ++c)
+            tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_tok_off[r] + j * BN);
+        } else {
+          const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
+          const int PR = min(BN, a.page_size);
+          for (int sb = 0; sb < BN / PR; ++sb) {
+            int t = j * BN + sb * PR;
+            if (t >= Lk) t = (Lk - 1) - ((Lk - 1) % PR);  // past the end: reload the last rows (masked)
+            int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + t / a.page_size];
+            if (page < 0 || page >= a.num_pages) {
+              set_status(a.status, FP2_DEV_PAGE_OOB);
+              page = 0;
+            }
+            const int flat = page * a.page_size + (t % a.page_size);
+            for (int c = 0; c < C::DCH; ++c)
+              tma_load_3d(dst + c * (BN * 128) + sb * (PR * 128), tm, &kv_full[slot], c * C::KCH, g, flat);
+          }
+        }
+      };
+      // Tiles whose loads go out before the mask exists: as many as fit in the ring without a
+      // release.  Their kept blocks come straight from the column list (clamped; the list is
+      // validated below and a bad one is reported through the status word).
+      const int npre = min(n_local, C::NSLOT / 2);
       if (lane == 0) {
         tma_prefetch_desc(&a.tm_q);
         tma_prefetch_desc(&a.tm_k);
@@ -269,6 +304,12 @@ __global__ void __launch_bounds__(384, 1)
               tma_load_3d(smem + C::OFF_Q + s * C::Q_BYTES + c * (128 * 128) + hs * (BN * 128), &a.tm_q, &q_full[s],
                           c * C::KCH, h, tokq);
           }
+        }
+        for (int t = 0; t < npre; ++t) {
+          const int jt = t_begin + t;
+          const int j = jt < n_virt ? -1 : min(max(a.col_idx[rs + jt - n_virt], 0), I);
+          issue_kv(jt, j, 2 * t, 0);
+          issue_kv(jt, j, 2 * t + 1, 1);
         }
       }
       const int nw = (I + 32) / 32;
@@ -290,11 +331,11 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(mask_ready);
         // Kept blocks are taken in ascending order from the bit mask in shared memory (the same
         // sequence as the validated column list), so the loop below makes no global reads for
-        // them.  A split starts after the kept blocks of the earlier splits.
+        // them.  It starts after the kept blocks of earlier splits and of the tiles issued above.
         const int nwords = (I >> 5) + 1;
         int wi = 0;
         uint32_t bits = kmask[0];
-        int skip = max(t_begin - n_virt, 0);
+        int skip = max(t_begin + npre - n_virt, 0);
         while (wi + 1 < nwords && skip >= __popc(bits)) {
           skip -= __popc(bits);
           bits = kmask[++wi];
@@ -307,10 +348,9 @@ __global__ void __launch_bounds__(384, 1)
           bits &= bits - 1;
           return j;
         };
-        int p = 0;
-        for (int jt = t_begin; jt < t_end && !*abort_flag; ++jt) {
-          int j = -1;
-          if (jt >= n_virt) j = next_kept();
+        int p = 2 * npre;
+        for (int jt = t_begin + npre; jt < t_end && !*abort_flag; ++jt) {
+          const int j = jt >= n_virt ? next_kept() : -1;
           bool stop = false;
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
@@ -318,32 +358,7 @@ __global__ void __launch_bounds__(384, 1)
               stop = true;
               break;
             }
-            mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
-            uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
-            if (j < 0) {
-              const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
-              for (int c = 0; c < C::DCH; ++c)
-                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_blk_off[r] + jt * BN);
-            } else if (a.page_table == nullptr) {
-              const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
-              for (int c = 0; c < C::DCH; ++c)
-                tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_tok_off[r] + j * BN);
-            } else {
-              const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
-              const int PR = min(BN, a.page_size);
-              for (int sb = 0; sb < BN / PR; ++sb) {
-                int t = j * BN + sb * PR;
-                if (t >= Lk) t = (Lk - 1) - ((Lk - 1) % PR);  // past the end: reload the last rows (masked)
-                int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + t / a.page_size];
-                if (page < 0 || page >= a.num_pages) {
-                  set_status(a.status, FP2_DEV_PAGE_OOB);
-                  page = 0;
-                }
-                const int flat = page * a.page_size + (t % a.page_size);
-                for (int c = 0; c < C::DCH; ++c)
-                  tma_load_3d(dst + c * (BN * 128) + sb * (PR * 128), tm, &kv_full[slot], c * C::KCH, g, flat);
-              }
-            }
+            issue_kv(jt, j, p, kv);
             ++p;
           }
           if (stop) break;
