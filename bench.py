@@ -37,7 +37,7 @@ FP8_WORKLOAD = "llama8b_128k_e4m3"
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
 # taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
-ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7252166912 + 1036569600, "source_sha": "cf93125e618cf4f1"}}
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7286387456 + 1057093888, "source_sha": "15a59014b75d9686"}}
 
 
 def source_sha(path):
