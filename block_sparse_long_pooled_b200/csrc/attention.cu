@@ -363,6 +363,21 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (stop) break;
         }
+        // The CTA that starts about one wave after this one (block index + grid SMs, in the
+        // heavy-first order) will need its Q tiles first: bring them into L2 now.
+        {
+          int r2, i2, sub2;
+          if (map_heavy_first(P, 1, a.Hkv * a.parts * a.splits, blockIdx.x + a.num_sms, r2, i2, sub2)) {
+            const int g2 = (sub2 / a.splits) / a.parts, part2 = (sub2 / a.splits) % a.parts;
+            constexpr int HS2 = 128 / BN;
+            for (int s = 0; s < a.NT; ++s)
+              for (int hs = 0; hs < HS2; ++hs) {
+                const int hl = (part2 * a.NT + s) * HS2 + hs;
+                for (int c = 0; c < C::DCH; ++c)
+                  tma_prefetch_l2_3d(&a.tm_q, c * C::KCH, g2 * a.G + (hl % a.G), P.tok_off[r2] + i2 * BN);
+              }
+          }
+        }
         // Never leave with copies in flight.
         for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status);
         for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status);

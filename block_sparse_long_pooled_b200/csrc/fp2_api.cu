@@ -386,6 +386,11 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   a.mean_correction = s->mean_correction ? 1 : 0;
   a.total_tokens = static_cast<int>(c.T);
   a.status = status_ptr(scratch);
+  {
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    a.num_sms = nsm;
+  }
   const int64_t items = c.total_blocks * p->num_kv_heads * a.parts * a.splits;
   if (items == 0) return FP2_OK;
   cudaError_t e = fp2::launch_attention(p->dtype, D, B, a, c.plan, items, st);

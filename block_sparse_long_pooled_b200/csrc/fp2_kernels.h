@@ -66,6 +66,7 @@ struct AttnArgs {
   int mean_correction;
   int total_tokens;
   int splits;                 // KV splits per row (1 = none)
+  int num_sms;                // SMs of the device (the launch's wave width)
   float* o_part;              // [splits, T, Hq, d] f32 partial outputs (splits > 1)
   float* lse_part;            // [splits, Hq, T] f32 partial LSE (splits > 1)
   uint32_t* status;
