@@ -19,6 +19,15 @@ namespace fp2 {
 
 constexpr int kJC = 32;  // key blocks per staged chunk
 
+FP2_DEVICE void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+FP2_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+FP2_DEVICE void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const Fp2Plan P) {
   extern __shared__ __align__(16) float smem[];
@@ -50,8 +59,8 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
 
   constexpr int KS = D + 4;  // padded pooled-key row (conflict-free float4 reads)
   float* qs = smem;                       // [TI*G][D]
-  float* ks = qs + a.TI * G * D;          // [kJC][KS]
-  float* sc = ks + kJC * KS;              // [TI*G][SP]
+  float* ks = qs + a.TI * G * D;          // [2][kJC][KS]: chunk being used, chunk in flight
+  float* sc = ks + 2 * kJC * KS;          // [TI*G][SP]
   float* thr = sc + a.TI * G * a.SP;      // [TI*G]
 
   for (int idx = tid; idx < rows * (D / 4); idx += 256) {
@@ -61,20 +70,35 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
         a.qbar)[(static_cast<int64_t>(bo + i0 + ii) * a.Hq + g * G + hl) * (D / 4) + c4];
   }
 
-  for (int j0 = 0; j0 < J1; j0 += kJC) {
-    __syncthreads();
+  // Key chunks are double-buffered with cp.async: chunk c+1 streams in while chunk c is used.
+  auto load_chunk = [&](int j0, int buf) {
+    float* kb = ks + buf * (kJC * KS);
     for (int idx = tid; idx < kJC * (D / 4); idx += 256) {
       const int jj = idx / (D / 4), c4 = idx % (D / 4);
       const int j = j0 + jj;
-      float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < J1) val = reinterpret_cast<const float4*>(a.kbar)[(static_cast<int64_t>(kbo + j) * a.Hkv + g) * (D / 4) + c4];
-      *reinterpret_cast<float4*>(&ks[jj * KS + c4 * 4]) = val;
+      float* dst = &kb[jj * KS + c4 * 4];
+      if (j < J1)
+        cp_async16(dst, &a.kbar[(static_cast<int64_t>(kbo + j) * a.Hkv + g) * D + c4 * 4]);
+      else
+        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
+    cp_async_commit();
+  };
+  load_chunk(0, 0);
+  for (int j0 = 0, it = 0; j0 < J1; j0 += kJC, ++it) {
+    const int buf = it & 1;
+    if (j0 + kJC < J1) {
+      load_chunk(j0 + kJC, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // chunk `buf` (and, on the first pass, the query rows) visible to all
+    const float* kb = ks + buf * (kJC * KS);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
     for (int k = 0; k < D; k += 4) {
-      const float4 kv = *reinterpret_cast<const float4*>(&ks[lane * KS + k]);
+      const float4 kv = *reinterpret_cast<const float4*>(&kb[lane * KS + k]);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int row = warp + 8 * u;
@@ -92,6 +116,7 @@ __global__ void __launch_bounds__(256) discover_kernel(const DiscArgs a, const F
       const int row = warp + 8 * u;
       if (row < rows && j0 + lane < J1) sc[row * a.SP + j0 + lane] = acc[u] * a.scale;
     }
+    __syncthreads();  // every thread is done with chunk `buf` before it is refilled
   }
   __syncthreads();
 
@@ -202,7 +227,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const uint32_t* __restrict
 }
 
 size_t discover_smem_bytes(int D, int G, int TI, int SP) {
-  return sizeof(float) * (static_cast<size_t>(TI) * G * D + kJC * (D + 4) + static_cast<size_t>(TI) * G * SP +
+  return sizeof(float) * (static_cast<size_t>(TI) * G * D + 2 * kJC * (D + 4) + static_cast<size_t>(TI) * G * SP +
                           static_cast<size_t>(TI) * G);
 }
 
