@@ -40,6 +40,22 @@ FP8_WORKLOAD = "llama8b_128k_e4m3"
 ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7286387456 + 1057093888, "source_sha": "15a59014b75d9686"}}
 
 
+def max_over_ranks(pg, x, device=None):
+    """The largest of x over all ranks of the process group (x itself when there is none)."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(flops_per_rank_step, world, ms_per_step):
+    """Whole-job throughput in TFLOP/s: every rank runs the same workload (weak scaling) and the
+    step time is the slowest rank's."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def source_sha(path):
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
@@ -587,10 +603,8 @@ def main():
     sampler.start()
     total_ms, stages = time_path(path, args.steps, args.warmup)
     clocks = sampler.stop()
+    total_ms = max_over_ranks(pg, total_ms, dev)
     if pg:
-        t = torch.tensor([total_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
         pg.barrier()
     st, bits = fp2.fp2_get_device_status(path.scratch)
     if st != fp2.FP2_OK:
@@ -598,7 +612,7 @@ def main():
     ms = total_ms / args.steps
     dense = w.dense_equiv_flops()
     ach, kept, pruned, causal = path.achieved_flops()
-    value = dense * world / (ms * 1e-3) / 1e12
+    value = whole_job_value(dense, world, ms)
     attn_tflops = ach / (stages["attend"] * 1e-3) / 1e12
     peak_bf16 = peaks["bf16_tflops_sustained"]
     peak = peak_bf16 if w.dtype != "e4m3" else 2.0 * peak_bf16
@@ -636,7 +650,8 @@ def main():
                             "attend_frac": dach / (dst["attend"] * 1e-3) / 1e12 / peak}
         del dense_path
         e2e_ms, serial_ms, h2d, d2h = time_e2e(path, max(4, args.steps // 5))
-        line["e2e"] = {"value": dense * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e_ms = max_over_ranks(pg, e2e_ms, dev)
+        line["e2e"] = {"value": whole_job_value(dense, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "mode": "pipelined: upload, fp2_prefill and download on three streams",
                        "serial_ms_per_step": serial_ms}
