@@ -60,11 +60,18 @@ struct AttnCfg {
   static constexpr int BM = 128;
   static constexpr int Q_BYTES = BM * D * ELT;
   static constexpr int KV_BYTES = BN * D * ELT;
+  // e4m3: QK runs on e4m3 operands; V tiles are converted to f16 in shared memory (exact) and PV
+  // runs as an f16 MMA with P written as f16.  V16 holds two converted tiles.
+  static constexpr bool V16 = DT == 2;
+  static constexpr int V16_BYTES = V16 ? BN * D * 2 : 0;
   static constexpr int TILE_BUDGET = 200 * 1024;
-  static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES) / KV_BYTES;
+  static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES - 2 * V16_BYTES) / KV_BYTES;
   static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
-  // P columns per M tile: one 32-bit column per key for f32, two keys per column for bf16,
-  // two e4m3 planes of four keys per column for e4m3.
+  // PV operand type: f16 for e4m3 inputs, else the input type; K extent of one PV MMA.
+  static constexpr int PV_KIND = V16 ? 1 : KIND;
+  static constexpr uint32_t PV_FMT = V16 ? 0u : FMT;  // kind::f16 format 0 = f16
+  static constexpr int PV_UK = V16 ? 16 : UK;
+  // P columns per M tile: one 32-bit column per key for f32, two keys per column for 16-bit P.
   static constexpr int PC = DT == 0 ? BN : BN / 2;
   static constexpr int S_COL = 0;
   static constexpr int P_COL0 = BN, P_COL1 = BN + PC;
@@ -76,16 +83,17 @@ struct AttnCfg {
   static_assert(128 * REG_LOW + 256 * REG_HIGH <= 384 * 168, "register split exceeds the launch");
   // Online-softmax constants (log2 domain).  P is written as 2^(x - m + P_SHIFT); the running
   // max m is only raised when the row max grows by more than LAZY, so P <= 2^(P_SHIFT + LAZY).
-  // e4m3: P_SHIFT 4 keeps small probabilities out of e4m3's subnormal range and 2^8 stays
-  // below its 448 maximum; P is then sent as two e4m3 terms (hi + lo).
+  // e4m3 inputs (P in f16): P_SHIFT 4 keeps small probabilities further from f16's subnormal
+  // range; 2^12 stays far below its 65504 maximum.
   static constexpr float P_SHIFT = DT == 2 ? 4.0f : 0.0f;
-  static constexpr float LAZY = DT == 2 ? 4.0f : 8.0f;
+  static constexpr float LAZY = 8.0f;
   static constexpr uint32_t IDESC_S = make_idesc(FMT, FMT, 0, 0, 128, BN);
-  static constexpr uint32_t IDESC_PV = make_idesc(FMT, FMT, 0, 1, 128, D);
+  static constexpr uint32_t IDESC_PV = make_idesc(PV_FMT, PV_FMT, 0, 1, 128, D);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2;
+  static constexpr int OFF_V16 = OFF_KV + NSLOT * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V16 + 2 * V16_BYTES;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 4;
   // Output staging for TMA stores: tile s's normalised O (128 rows x d, output type) goes into
   // the shared memory of its own Q tile, free once the tile's last QK product is done; only when
   // it fits there (bf16 and f32 inputs; e4m3 Q tiles are half the size of a bf16 O tile).
@@ -189,6 +197,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* s_free = mma_done + 1;  // [2]: the S buffer has been copied out by softmax s
   uint64_t* pv_done = s_free + 2;   // the PV issuer's final commit
   uint64_t* o_staged = pv_done + 1; // [2]: every row of tile s is staged for the TMA store
+  uint64_t* v16_full = o_staged + 2;   // [2]: converted f16 V tile ready (e4m3 inputs)
+  uint64_t* v16_empty = v16_full + 2;  // [2]: its PV products are done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
@@ -228,6 +238,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&o_done[s], 1);
       mbar_init(&s_free[s], 128);
       mbar_init(&o_staged[s], 128);
+      mbar_init(&v16_full[s], 1);
+      mbar_init(&v16_empty[s], 1);
     }
     for (int k = 0; k < C::NSLOT; ++k) {
       mbar_init(&kv_full[k], 1);
@@ -449,34 +461,79 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t pcol = tmem + (s ? C::P_COL1 : C::P_COL0);
             const uint32_t ocol = tmem + (s ? C::O_COL1 : C::O_COL0);
             // V is MN-major (d contiguous).  32-bit V uses the 32-byte-chunk swizzle with 4-row
-            // atoms (SBO 512); 16/8-bit V the 16-byte-chunk swizzle with 8-row atoms.
+            // atoms (SBO 512); 16-bit V the 16-byte-chunk swizzle with 8-row atoms.
             const uint64_t vd0 = DT == 0 ? smem_desc(vaddr, BN * 128, 512, 1u) : smem_desc_sw128(vaddr, BN * 128, 1024);
 #pragma unroll 1
-            for (int k = 0; k < BN / C::UK; ++k) {
-              const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::UK * 128) >> 4);
-              if constexpr (DT == 2) {
-                umma_ts_warp<C::KIND>(ocol, pcol + k * 16, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-                umma_ts_warp<C::KIND>(ocol, pcol + k * 16 + 8, bd, C::IDESC_PV, 1u);
-              } else {
-                umma_ts_warp<C::KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
-              }
+            for (int k = 0; k < BN / C::PV_UK; ++k) {
+              const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::PV_UK * 128) >> 4);
+              umma_ts_warp<C::PV_KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
             }
             umma_commit_warp(&o_done[s]);
           };
           for (int jt = 0; jt < n_local && ok; ++jt) {
             const int qv = 2 * jt + 1;
-            if (!kv_wait(qv)) break;
+            uint32_t vaddr;
+            if constexpr (C::V16) {
+              if (!(ok = wait_all(&v16_full[jt & 1], (jt >> 1) & 1))) break;
+              vaddr = sbase + C::OFF_V16 + (jt & 1) * C::V16_BYTES;
+            } else {
+              if (!(ok = kv_wait(qv))) break;
+              vaddr = slot_addr(qv);
+            }
             for (int s = 0; s < a.NT; ++s) {
               if (!(ok = wait_all(&p_full[s], jt & 1))) break;
               tc_fence_after();
-              issue_pv(s, slot_addr(qv), jt);
+              issue_pv(s, vaddr, jt);
             }
             if (!ok) break;
-            umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
+            if constexpr (C::V16)
+              umma_commit_warp(&v16_empty[jt & 1]);  // converted V(jt) fully consumed
+            else
+              umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
           }
           umma_commit_warp(pv_done);
           if (lane == 0) mbar_wait_drain(pv_done, 0, a.status);
           __syncwarp();
+        }
+      }
+    } else if (warp == 11) {
+      if constexpr (C::V16) {
+        // ---------------------------------------------------------------- V converter (e4m3)
+        // Each V tile (BN keys x 128 e4m3, 128-byte swizzled rows) becomes an f16 tile in the
+        // layout the PV MMA reads (two 64-column chunks of BN rows x 128 bytes, swizzled); exact,
+        // since every e4m3 value is an f16 value.  The ring slot is released once it is read.
+        // Source row j: 16-byte unit u holds d 16u .. 16u+15 at position u ^ (j & 7).
+        // Destination chunk c, row j: 16-byte unit u holds d 64c + 8u .. +7 at position u ^ (j & 7).
+        static_assert(D == 128, "the e4m3 V converter assumes d = 128");
+        bool ok = true;
+        for (int jt = 0; jt < n_local && ok; ++jt) {
+          const int qv = 2 * jt + 1, slot = qv % C::NSLOT;
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&kv_full[slot], (qv / C::NSLOT) & 1, abort_flag, a.status));
+          if (ok && jt >= 2)
+            ok = __all_sync(0xFFFFFFFFu,
+                            mbar_wait(&v16_empty[jt & 1], ((jt >> 1) - 1) & 1, abort_flag, a.status));
+          if (!ok) break;
+          const uint8_t* src = smem + C::OFF_KV + slot * C::KV_BYTES;
+          uint8_t* dst = smem + C::OFF_V16 + (jt & 1) * C::V16_BYTES;
+  #pragma unroll 2
+          for (int x = lane; x < BN * 8; x += 32) {
+            const int j = x >> 3, u = x & 7;
+            const uint4 w = *reinterpret_cast<const uint4*>(src + j * 128 + ((u ^ (j & 7)) << 4));
+            const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x & 0xFFFFu), e4m3x2_to_f16x2(w.x >> 16),
+                                        e4m3x2_to_f16x2(w.y & 0xFFFFu), e4m3x2_to_f16x2(w.y >> 16));
+            const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z & 0xFFFFu), e4m3x2_to_f16x2(w.z >> 16),
+                                        e4m3x2_to_f16x2(w.w & 0xFFFFu), e4m3x2_to_f16x2(w.w >> 16));
+            const int c = u >> 2, u0 = 2 * (u & 3);
+            uint8_t* rowp = dst + c * (BN * 128) + j * 128;
+            *reinterpret_cast<uint4*>(rowp + ((u0 ^ (j & 7)) << 4)) = lo;
+            *reinterpret_cast<uint4*>(rowp + (((u0 + 1) ^ (j & 7)) << 4)) = hi;
+          }
+          fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&kv_empty[slot]);
+            mbar_arrive(&v16_full[jt & 1]);
+          }
         }
       }
     }
@@ -614,22 +671,17 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(p_addr + c * 32, pk);
           }
         } else if constexpr (DT == 2) {
-          // K-step c (32 keys) of the PV MMA: hi plane at columns [16c, 16c+8), lo at [16c+8, 16c+16);
-          // two K-steps (32 words) per TMEM store.
+          // f16 P for the f16 PV product: 64 scores -> 32 packed words -> one TMEM store.
   #pragma unroll
-          for (int h = 0; h < BN / 64; ++h) {
+          for (int c = 0; c < BN / 64; ++c) {
             uint32_t pk[32];
   #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-  #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const int c = 2 * h + cc;
-                const float2 pa = exp_pair(c * 16 + 2 * e), pb = exp_pair(c * 16 + 2 * e + 1);
-                split_e4m3x4(pa.x, pa.y, pb.x, pb.y, pk[cc * 16 + e], pk[cc * 16 + 8 + e]);
-              }
+            for (int e = 0; e < 32; ++e) {
+              const float2 p = exp_pair(c * 32 + e);
+              pk[e] = pack_f16x2(p.x, p.y);
             }
-            if (h == 0 && !wait_pv_prev()) break;
-            tmem_st32(p_addr + h * 32, pk);
+            if (c == 0 && !wait_pv_prev()) break;
+            tmem_st32(p_addr + c * 32, pk);
           }
         } else {
           uint32_t pk[BN];

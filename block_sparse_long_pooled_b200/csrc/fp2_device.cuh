@@ -372,22 +372,19 @@ FP2_DEVICE uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// e4m3x2 (low byte = first value) -> two floats, exact.
-FP2_DEVICE float2 e4m3x2_to_float2(uint16_t v) {
+// Two floats -> packed f16x2 (lo in the low half).
+FP2_DEVICE uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// e4m3x2 (low byte = first value) -> f16x2 bits (first value in the low half), exact.
+FP2_DEVICE uint32_t e4m3x2_to_f16x2(uint32_t v16) {
   uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(v16)));
+  return h;
 }
 
-// Two-term e4m3 split of four values: hi = e4m3(v), lo = e4m3(v - hi), packed 4 per word.
-// hi + lo carries about 7 significant bits instead of 4.
-FP2_DEVICE void split_e4m3x4(float v0, float v1, float v2, float v3, uint32_t& hi, uint32_t& lo) {
-  uint16_t h01, h23;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h01) : "f"(v1), "f"(v0));
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h23) : "f"(v3), "f"(v2));
-  const float2 b01 = e4m3x2_to_float2(h01), b23 = e4m3x2_to_float2(h23);
-  hi = static_cast<uint32_t>(h01) | (static_cast<uint32_t>(h23) << 16);
-  lo = pack_e4m3x4(v0 - b01.x, v1 - b01.y, v2 - b23.x, v3 - b23.y);
-}
+
 
 }  // namespace fp2
