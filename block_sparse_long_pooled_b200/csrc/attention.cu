@@ -21,17 +21,21 @@
 //   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S (and
 //                    release the S buffer at once), mask, online max with lazy O rescale
 //                    (only when the running max grows past a threshold), write P (bf16, f32,
-//                    or e4m3 as a hi + lo pair of planes) to the tile's P columns in TMEM, and
-//                    finally normalise O and store it.
-//   warp 8           producer: builds the kept-block bitmask, issues TMA loads of Q once and
-//                    of K/V (or kbar/vbar) tiles into an NSLOT ring of shared-memory slots.
+//                    or f16 for e4m3 inputs) to the tile's P columns in TMEM, and finally
+//                    normalise O and write it (full blocks through a swizzled staging tile and
+//                    TMA stores, partial blocks and KV-split partials with per-thread stores).
+//   warp 8           producer: issues TMA loads of Q and the first key tiles, builds the
+//                    kept-block bitmask, then loads the remaining K/V (or kbar/vbar) tiles into
+//                    an NSLOT ring of shared-memory slots; finally prefetches into L2 the Q tiles
+//                    of the CTA one wave ahead.
 //   warp 9           QK issuer: S = Q_s K^T (SS form) into the shared S buffer.
 //   warp 10          PV issuer: O_s += P_s V (A operand P_s read from TMEM).  The two products
 //                    touch disjoint TMEM, so each is issued the moment its own inputs are ready
 //                    and the tensor pipe interleaves them; one issuer would stall the pipe at
 //                    every wait between groups.  Both issue tcgen05.mma from lane 0 and signal
 //                    mbarriers with tcgen05.commit.
-//   warp 11          idle (it completes warpgroup 2 for the register split).
+//   warp 11          e4m3 inputs: converts each V tile to f16 in shared memory for the f16 PV
+//                    product; otherwise idle (it completes warpgroup 2 for the register split).
 // TMEM: S | P0 | P1 | O0 | O1.  One S buffer serves both M tiles in turn: a softmax warpgroup
 // copies its S tile into registers and releases the buffer before doing any arithmetic, so
 // the next QK product (the other tile's, or this tile's next key tile) is computed while the
