@@ -37,7 +37,7 @@ FP8_WORKLOAD = "llama8b_128k_e4m3"
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
 # taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
-ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7286387456 + 1057093888, "source_sha": "15a59014b75d9686"}}
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7606532352 + 1058762752, "source_sha": "37c8408d6b14c538"}}
 
 
 def max_over_ranks(pg, x, device=None):
