@@ -197,6 +197,12 @@ class Path:
         d, B = w.head_dim, w.block_size
         return 4.0 * d * B * B * kept + 4.0 * d * B * pruned, kept, pruned, causal
 
+    def discover_flops(self):
+        """Algorithmic flops of the pooled block scores: 2 d per (q head, query block, causal key block)."""
+        w = self.w
+        nb = [-(-L // w.block_size) for L in w.seqlens]
+        return 2.0 * w.head_dim * w.num_q_heads * sum(n * (n + 1) // 2 for n in nb)
+
     def pool_bytes(self):
         w = self.w
         elt = {"f32": 4, "bf16": 2, "e4m3": 1}[w.dtype]
@@ -205,6 +211,13 @@ class Path:
         read = T * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * elt
         write = nb * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * 4 + 2 * nb * w.num_kv_heads * w.head_dim * elt
         return read + write
+
+
+def fp32_fma_peak_tflops(clocks):
+    """fp32 CUDA-core peak of a B200 from its unit counts: 148 SMs x 128 FMA lanes per clock x 2
+    flops at the maximum SM clock (packed f32x2 FMAs issue at the same lane rate)."""
+    mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
 
 
 def time_path(path, steps, warmup):
@@ -637,6 +650,12 @@ def main():
         "pool_roofline": {"bound": "hbm", "achieved": path.pool_bytes() / (stages["pool"] * 1e-3) / 1e9,
                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": path.pool_bytes() / (stages["pool"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "discover_roofline": {"bound": "alu", "achieved": path.discover_flops() / (stages["discover"] * 1e-3) / 1e12,
+                              "peak": fp32_fma_peak_tflops(clocks), "unit": "TFLOP/s",
+                              "frac": path.discover_flops() / (stages["discover"] * 1e-3) / 1e12
+                              / fp32_fma_peak_tflops(clocks),
+                              "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 flops x max SM clock (unit counts)",
+                              "includes": "discover_kernel + scan_kernel + scatter_kernel"},
         "clocks": clocks,
         "gpu_launches": 5 * args.steps,
     }
