@@ -145,6 +145,32 @@ def test_full_size_workloads(name):
         assert 0.04 <= stats["density"] <= 0.06
 
 
+# More than 1024 key blocks: 32 score rows of a tile no longer fit in shared memory, so discovery
+# runs with smaller query tiles (the library picks 24, 16 and 8 rows here) and part of its warps
+# have no row; the last case is the largest sequence the ABI accepts (FP2_MAX_BLOCKS = 4096).
+LONG = [
+    small("long_g4_tile24", num_q_heads=4, num_kv_heads=1, head_dim=64, block_size=64, seqlens=(1400 * 64 - 17,),
+          sink_blocks=2, window_blocks=4),
+    small("long_g8_tile16", num_q_heads=8, num_kv_heads=1, head_dim=64, block_size=64, seqlens=(2100 * 64 + 5,),
+          sink_blocks=2, window_blocks=4),
+    small("long_g4_max_blocks", num_q_heads=4, num_kv_heads=1, head_dim=64, block_size=64, seqlens=(4096 * 64,),
+          sink_blocks=2, window_blocks=4),
+]
+
+
+@pytest.mark.parametrize("w", LONG, ids=lambda w: w.name)
+def test_long_sequences_smaller_discovery_tiles(w):
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp, head_chunk=4)
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), lse=False)
+    Hn.compare_pooled(run, inp, ora)
+    stats = Hn.compare_index(run, inp, ora)
+    print(f"{w.name}: density {stats['density']*100:.2f}%  borderline {stats['borderline_blocks']} "
+          f"mismatched {stats['borderline_mismatches']}")
+    Hn.compare_attention_sampled(run, inp, ora, n_per_seq=32)
+
+
 def test_page_table_out_of_range_is_reported_not_faulted():
     """A corrupt page id is clamped on the device and reported through the status word."""
     import torch
