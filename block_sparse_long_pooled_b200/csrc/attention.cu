@@ -97,7 +97,7 @@ struct AttnCfg {
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_V16 = OFF_KV + NSLOT * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V16 + 2 * V16_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 4;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 4 + 2;
   // Output staging for TMA stores: tile s's normalised O (128 rows x d, output type) goes into
   // the shared memory of its own Q tile, free once the tile's last QK product is done; only when
   // it fits there (bf16 and f32 inputs; e4m3 Q tiles are half the size of a bf16 O tile).
@@ -203,19 +203,40 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_staged = pv_done + 1; // [2]: every row of tile s is staged for the TMA store
   uint64_t* v16_full = o_staged + 2;   // [2]: converted f16 V tile ready (e4m3 inputs)
   uint64_t* v16_empty = v16_full + 2;  // [2]: its PV products are done
+  uint64_t* o_merge = v16_empty + 2;   // [2]: piece CTAs: the tile's merge decision is in merge_flag
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
   uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int r, i, sub;
-  if (!map_heavy_first(P, 1, a.Hkv * a.parts * a.splits, blockIdx.x, r, i, sub)) return;
-  const int split = sub % a.splits;
-  const int g = (sub / a.splits) / a.parts, part = (sub / a.splits) % a.parts;
+  // CTAs [0, a.adapt) run the planned pieces of long rows (adaptive splits); the rest map to
+  // (sequence, query block, KV head, part, split) in heavy-first order.
+  int r, i, g, part, split, nsplit;
+  const int item = static_cast<int>(blockIdx.x) < a.adapt ? static_cast<int>(blockIdx.x) : -1;
+  if (item >= 0) {
+    if (item >= *a.n_items) return;
+    const int2 it = a.items[item];
+    const int b = it.x / a.Hkv;
+    g = it.x % a.Hkv;
+    r = seq_of_block(P, b);
+    i = b - P.blk_off[r];
+    nsplit = it.y >> 16;
+    part = (it.y >> 8) & 255;
+    split = it.y & 255;
+  } else {
+    int sub;
+    if (!map_heavy_first(P, 1, a.Hkv * a.parts * a.splits, blockIdx.x - a.adapt, r, i, sub)) return;
+    nsplit = a.splits;
+    split = sub % a.splits;
+    g = (sub / a.splits) / a.parts;
+    part = (sub / a.splits) % a.parts;
+  }
   const int L = P.len[r];                 // query tokens of the sequence (or chunk)
   const int I = P.pre_blk[r] + i;         // absolute key block of query block i (the diagonal)
   const int Lk = P.pre_blk[r] * BN + L;   // key tokens of the sequence
   const int64_t row = static_cast<int64_t>(P.blk_off[r] + i) * a.Hkv + g;
+  if (item < 0 && a.adapt > 0 && a.row_item0[row] >= 0) return;  // this row runs as pieces
   const int rs = a.row_ptr[row], re = a.row_ptr[row + 1];
   const int nkept = re - rs;
   if (nkept <= 0 || nkept > I + 1) {
@@ -226,8 +247,8 @@ __global__ void __launch_bounds__(384, 1)
   const int n_virt = (a.mean_correction && npruned > 0) ? (I + BN - 1) / BN : 0;
   const int n_tiles = n_virt + nkept;
   // Count-balanced KV split: this CTA takes key tiles [t_begin, t_end) of the row's stream.
-  const int t_begin = static_cast<int>(static_cast<long long>(n_tiles) * split / a.splits);
-  const int t_end = static_cast<int>(static_cast<long long>(n_tiles) * (split + 1) / a.splits);
+  const int t_begin = static_cast<int>(static_cast<long long>(n_tiles) * split / nsplit);
+  const int t_end = static_cast<int>(static_cast<long long>(n_tiles) * (split + 1) / nsplit);
   const int n_local = t_end - t_begin;
 
   if (warp == 0) {
@@ -244,6 +265,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&o_staged[s], 128);
       mbar_init(&v16_full[s], 1);
       mbar_init(&v16_empty[s], 1);
+      mbar_init(&o_merge[s], 1);
     }
     for (int k = 0; k < C::NSLOT; ++k) {
       mbar_init(&kv_full[k], 1);
@@ -383,7 +405,8 @@ __global__ void __launch_bounds__(384, 1)
         // heavy-first order) will need its Q tiles first: bring them into L2 now.
         {
           int r2, i2, sub2;
-          if (map_heavy_first(P, 1, a.Hkv * a.parts * a.splits, blockIdx.x + a.num_sms, r2, i2, sub2)) {
+          const long long v2 = static_cast<long long>(blockIdx.x) + a.num_sms - a.adapt;
+          if (v2 >= 0 && map_heavy_first(P, 1, a.Hkv * a.parts * a.splits, v2, r2, i2, sub2)) {
             const int g2 = (sub2 / a.splits) / a.parts, part2 = (sub2 / a.splits) % a.parts;
             constexpr int HS2 = 128 / BN;
             for (int s = 0; s < a.NT; ++s)
@@ -711,7 +734,95 @@ __global__ void __launch_bounds__(384, 1)
       if (ok && done_tiles == n_local && n_local > 0)
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_local - 1) & 1, abort_flag, a.status));
       tc_fence_after();
-      if (ok && a.splits > 1) {
+      if (item >= 0) {
+        // Piece of a split row: its normalised partial O (fp32) and natural-log LSE go to the
+        // piece's slot; the last piece of the (row, part) to finish, found with an atomic counter
+        // per M tile, merges all of them with weights exp(LSE - max LSE) and writes the output
+        // rows.  No CTA waits for another.  A piece with no visible key contributes LSE = -inf.
+        const int prow = a.NT * 128;
+        const int64_t srow = static_cast<int64_t>(item) * prow + s * 128 + rt;
+        const bool any = ok && n_local > 0 && l_run > 0.f;
+        const float inv = any ? a.v_descale / l_run : 0.f;
+        float* op = a.o_slot + srow * D;
+  #pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (ok && n_local > 0) {
+            tmem_ld32_sync(o_addr + c * 32, v);
+          } else {
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          float4* dst = reinterpret_cast<float4*>(op + c * 32);
+  #pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                 __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+        }
+        a.lse_slot[srow] = any ? (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f : -CUDART_INF_F;
+        __threadfence();
+        mbar_arrive(&o_staged[s]);
+        const int first = item - split;  // first piece of this (row, part)
+        if (qd == 0 && lane == 0) {
+          int last = 0;
+          if (mbar_wait(&o_staged[s], 0, abort_flag, a.status)) {
+            __threadfence();
+            last = atomicAdd(&a.piece_cnt[first * 2 + s], 1) == nsplit - 1;
+          }
+          merge_flag[s] = last;
+          mbar_arrive(&o_merge[s]);
+        }
+        const bool merge =
+            __all_sync(0xFFFFFFFFu, mbar_wait(&o_merge[s], 0, abort_flag, a.status)) && merge_flag[s] != 0;
+        if (merge && row_ok) {
+          __threadfence();
+          const float* lp = a.lse_slot + static_cast<int64_t>(first) * prow + s * 128 + rt;
+          const float* obase = a.o_slot + (static_cast<int64_t>(first) * prow + s * 128 + rt) * D;
+          float m = -CUDART_INF_F;
+          for (int k = 0; k < nsplit; ++k) m = fmaxf(m, __ldcg(lp + static_cast<int64_t>(k) * prow));
+          float wsum = 0.f;
+          for (int k = 0; k < nsplit; ++k) {
+            const float l = __ldcg(lp + static_cast<int64_t>(k) * prow);
+            wsum += l == -CUDART_INF_F ? 0.f : expf(l - m);
+          }
+          const float winv = wsum > 0.f ? 1.f / wsum : 0.f;
+          const int tok = P.tok_off[r] + i * BN + tl;
+  #pragma unroll 1
+          for (int c = 0; c < D / 8; ++c) {  // eight output columns at a time
+            float acc8[8];
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) acc8[e] = 0.f;
+            for (int k = 0; k < nsplit; ++k) {
+              const float l = __ldcg(lp + static_cast<int64_t>(k) * prow);
+              const float w = l == -CUDART_INF_F ? 0.f : expf(l - m);
+              const float4* src = reinterpret_cast<const float4*>(obase + static_cast<int64_t>(k) * prow * D + c * 8);
+              const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+              acc8[0] = fmaf(w, x0.x, acc8[0]);
+              acc8[1] = fmaf(w, x0.y, acc8[1]);
+              acc8[2] = fmaf(w, x0.z, acc8[2]);
+              acc8[3] = fmaf(w, x0.w, acc8[3]);
+              acc8[4] = fmaf(w, x1.x, acc8[4]);
+              acc8[5] = fmaf(w, x1.y, acc8[5]);
+              acc8[6] = fmaf(w, x1.z, acc8[6]);
+              acc8[7] = fmaf(w, x1.w, acc8[7]);
+            }
+            const int64_t o_off = (static_cast<int64_t>(tok) * a.Hq + h) * D + c * 8;
+            if constexpr (DT == 0) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + o_off);
+              dst[0] = make_float4(acc8[0] * winv, acc8[1] * winv, acc8[2] * winv, acc8[3] * winv);
+              dst[1] = make_float4(acc8[4] * winv, acc8[5] * winv, acc8[6] * winv, acc8[7] * winv);
+            } else {
+              uint4 w;
+              w.x = pack_bf16x2(acc8[0] * winv, acc8[1] * winv);
+              w.y = pack_bf16x2(acc8[2] * winv, acc8[3] * winv);
+              w.z = pack_bf16x2(acc8[4] * winv, acc8[5] * winv);
+              w.w = pack_bf16x2(acc8[6] * winv, acc8[7] * winv);
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o_off) = w;
+            }
+          }
+          if (a.lse != nullptr) a.lse[static_cast<int64_t>(h) * a.total_tokens + tok] = m + logf(wsum);
+        }
+      } else if (ok && a.splits > 1) {
         // Partial result of this split: normalised O (fp32) and its natural-log LSE, merged by
         // combine_kernel.  A split with no key tile (or no visible key for this row) contributes
         // O = 0 with LSE = -inf.
@@ -828,6 +939,98 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// Adaptive count-balanced splits (paper page, Table 7: "count-balanced CSR splits"), planned on
+// the device from the index, so the host needs no copy of it.  One CTA sizes every row in key
+// tiles as the attention kernel streams them (virtual tiles of the mean correction + kept
+// blocks), picks the piece size T (piece_tiles, or the launch's total tile work over 4 x SMs, at
+// least 32), and lists min(64, ceil(tiles / T)) pieces for every part of each row longer than T,
+// rows in index order, while they fit in a.adapt.  The pieces of one (row, part) are consecutive.
+__global__ void __launch_bounds__(1024) split_plan_kernel(const __grid_constant__ AttnArgs a,
+                                                          const __grid_constant__ Fp2Plan P, int64_t rows, int BN,
+                                                          int piece_tiles) {
+  __shared__ long long red[32];
+  __shared__ int n_used;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t seg = (rows + 1023) / 1024;
+  const int64_t s0 = min(rows, tid * seg), s1 = min(rows, s0 + seg);
+  const int r_first = s0 < rows ? seq_of_block(P, static_cast<int>(s0 / a.Hkv)) : 0;
+  auto row_tiles = [&](int64_t x, int& rc) {
+    const int b = static_cast<int>(x / a.Hkv);
+    while (rc + 1 < P.num_seqs && P.blk_off[rc + 1] <= b) ++rc;
+    const int I = P.pre_blk[rc] + (b - P.blk_off[rc]);
+    const int nk = max(0, min(a.row_ptr[x + 1] - a.row_ptr[x], I + 1));
+    const int nv = (a.mean_correction && I + 1 - nk > 0) ? (I + BN - 1) / BN : 0;
+    return nv + nk;
+  };
+  // Block sum of one value per thread (every thread gets the total).
+  auto block_sum = [&](long long v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    long long t = 0;
+    for (int w = 0; w < 32; ++w) t += red[w];
+    __syncthreads();
+    return t;
+  };
+  for (int k = tid; k < a.adapt * 2; k += 1024) a.piece_cnt[k] = 0;
+  if (tid == 0) n_used = 0;
+  long long T = piece_tiles;
+  if (T <= 0) {
+    long long loc = 0;
+    int rc = r_first;
+    for (int64_t x = s0; x < s1; ++x) loc += row_tiles(x, rc);
+    const long long slots = 4LL * max(a.num_sms, 1);
+    T = max(32LL, (block_sum(loc) * a.parts + slots - 1) / slots);
+  }
+  auto pieces_of = [&](int t) { return t > T ? static_cast<int>(min(64LL, (t + T - 1) / T)) : 1; };
+  // Exclusive scan of the piece counts (pieces x parts of each split row) over the rows.
+  long long loc = 0;
+  {
+    int rc = r_first;
+    for (int64_t x = s0; x < s1; ++x) {
+      const int S = pieces_of(row_tiles(x, rc));
+      if (S > 1) loc += static_cast<long long>(S) * a.parts;
+    }
+  }
+  long long incl = loc;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) red[warp] = incl;
+  __syncthreads();
+  long long before = 0;
+  for (int w = 0; w < warp; ++w) before += red[w];
+  long long base = before + incl - loc;
+  int rc = r_first;
+  int used = 0;
+  for (int64_t x = s0; x < s1; ++x) {
+    const int S = pieces_of(row_tiles(x, rc));
+    const long long cnt = S > 1 ? static_cast<long long>(S) * a.parts : 0;
+    if (cnt > 0 && base + cnt <= a.adapt) {
+      a.row_item0[x] = static_cast<int32_t>(base);
+      for (int pt = 0; pt < a.parts; ++pt)
+        for (int k = 0; k < S; ++k)
+          a.items[base + pt * S + k] = make_int2(static_cast<int>(x), (S << 16) | (pt << 8) | k);
+      used = static_cast<int>(base + cnt);
+    } else {
+      a.row_item0[x] = -1;
+    }
+    base += cnt;
+  }
+  atomicMax(&n_used, used);
+  __syncthreads();
+  if (tid == 0) *a.n_items = n_used;
+}
+
+cudaError_t launch_split_plan(const AttnArgs& a, const Fp2Plan& P, int64_t rows, int B, int piece_tiles,
+                              cudaStream_t stream) {
+  split_plan_kernel<<<1, 1024, 0, stream>>>(a, P, rows, B, piece_tiles);
+  return cudaGetLastError();
 }
 
 // Merge of the KV-split partials: for every (token, head), O = sum_s w_s O_s / sum_s w_s and

@@ -30,6 +30,10 @@ fp2_status cuda_fail(cudaError_t e, const char* what) {
 
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+// Adaptive splits: at most kMaxPieces pieces per attention launch (the automatic rule typically
+// plans 2-3 x SMs), and at most kMaxPieceSplits pieces per row.
+constexpr int kMaxPieces = 768;
+constexpr int kMaxPieceSplits = 64;
 
 int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : (t == FP2_BF16 ? 2 : 1); }
 
@@ -43,6 +47,9 @@ struct Ctx {
   size_t off_bitmask = 0, off_counts = 0;  // inside scratch
   int NT = 1, parts = 1, splits = 1;        // attention launch shape
   size_t off_opart = 0, off_lsepart = 0;    // KV-split partials inside scratch (splits > 1)
+  // Adaptive splits (splits == 1): up to `pieces` pieces of long rows, planned on the device.
+  int pieces = 0, piece_tiles = 0;          // piece capacity; forced piece size (0 = automatic)
+  size_t off_item0 = 0, off_items = 0, off_nitems = 0, off_pcnt = 0, off_oslot = 0, off_lslot = 0;
   // fp2_prefill carve-outs (offsets after scratch_bytes)
   size_t off_qbar = 0, off_kbar = 0, off_vbar = 0, off_kbm = 0, off_vbm = 0, off_rowptr = 0, off_colidx = 0;
 };
@@ -67,7 +74,8 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   if (!(s->alpha >= 0.f && s->alpha <= 1.f)) return fail(FP2_ERR_INVALID_ARG, "alpha must be in [0, 1]");
   if (s->sink_blocks < 0 || s->window_blocks < 0 || s->last_n_blocks < 0 || s->min_sparse_len < 0)
     return fail(FP2_ERR_INVALID_ARG, "sink/window/last_n/min_sparse_len must be >= 0");
-  if (s->kv_splits < 0 || s->kv_splits > 64) return fail(FP2_ERR_INVALID_ARG, "kv_splits must be in [0, 64]");
+  if (s->kv_splits < -FP2_MAX_BLOCKS || s->kv_splits > 64)
+    return fail(FP2_ERR_INVALID_ARG, "kv_splits must be in [-FP2_MAX_BLOCKS, 64]");
   if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale))
     return fail(FP2_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   for (float d : {p->q_descale, p->k_descale, p->v_descale})
@@ -170,9 +178,17 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   const int64_t row_ctas = c.rows * c.parts;
   if (s->kv_splits > 0)
     c.splits = s->kv_splits;
+  else if (s->kv_splits < 0)
+    c.splits = 1;
   else
     c.splits = row_ctas >= 296 ? 1 : static_cast<int>(std::min<int64_t>(8, (296 + std::max<int64_t>(row_ctas, 1) - 1) /
                                                                                    std::max<int64_t>(row_ctas, 1)));
+  // Rows whose key-tile count is far above the launch's share per SM are cut into pieces planned
+  // on the device (kv_splits < 0: pieces of at most -kv_splits tiles; 0 with many rows: automatic).
+  if (c.splits == 1 && s->kv_splits <= 0) {
+    c.piece_tiles = s->kv_splits < 0 ? -s->kv_splits : 0;
+    c.pieces = static_cast<int>(std::min<int64_t>(kMaxPieces, row_ctas * kMaxPieceSplits));
+  }
   c.off_bitmask = FP2_SCRATCH_STATUS_BYTES;
   c.off_counts = c.off_bitmask + align_up(static_cast<size_t>(c.rows) * c.W * 4);
   w.scratch_bytes = c.off_counts + align_up(static_cast<size_t>(c.rows) * 4);
@@ -181,6 +197,16 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
     c.off_opart = w.scratch_bytes;
     c.off_lsepart = c.off_opart + align_up(static_cast<size_t>(c.splits) * T * Hq * D * 4);
     w.scratch_bytes = c.off_lsepart + align_up(static_cast<size_t>(c.splits) * Hq * T * 4);
+  }
+  if (c.pieces > 0) {
+    const size_t prow = static_cast<size_t>(c.NT) * 128;  // packed rows of one piece
+    c.off_item0 = w.scratch_bytes;
+    c.off_items = c.off_item0 + align_up(static_cast<size_t>(c.rows) * 4);
+    c.off_nitems = c.off_items + align_up(static_cast<size_t>(c.pieces) * 8);
+    c.off_pcnt = c.off_nitems + align_up(4);
+    c.off_oslot = c.off_pcnt + align_up(static_cast<size_t>(c.pieces) * 2 * 4);
+    c.off_lslot = c.off_oslot + align_up(static_cast<size_t>(c.pieces) * prow * D * 4);
+    w.scratch_bytes = c.off_lslot + align_up(static_cast<size_t>(c.pieces) * prow * 4);
   }
   size_t o = w.scratch_bytes;
   c.off_qbar = o;   o += align_up(w.qbar_bytes);
@@ -379,6 +405,14 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   a.splits = c.splits;
   a.o_part = c.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(scratch) + c.off_opart) : nullptr;
   a.lse_part = c.splits > 1 ? reinterpret_cast<float*>(static_cast<char*>(scratch) + c.off_lsepart) : nullptr;
+  char* sc = static_cast<char*>(scratch);
+  a.adapt = c.pieces;
+  a.row_item0 = c.pieces ? reinterpret_cast<int32_t*>(sc + c.off_item0) : nullptr;
+  a.items = c.pieces ? reinterpret_cast<int2*>(sc + c.off_items) : nullptr;
+  a.n_items = c.pieces ? reinterpret_cast<int32_t*>(sc + c.off_nitems) : nullptr;
+  a.piece_cnt = c.pieces ? reinterpret_cast<int32_t*>(sc + c.off_pcnt) : nullptr;
+  a.o_slot = c.pieces ? reinterpret_cast<float*>(sc + c.off_oslot) : nullptr;
+  a.lse_slot = c.pieces ? reinterpret_cast<float*>(sc + c.off_lslot) : nullptr;
   a.sm_scale_log2 = static_cast<float>(static_cast<double>(c.scale) * 1.4426950408889634 *
                                        static_cast<double>(p->q_descale) * static_cast<double>(p->k_descale));
   a.v_descale = p->v_descale;
@@ -391,9 +425,14 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
     a.num_sms = nsm;
   }
-  const int64_t items = c.total_blocks * p->num_kv_heads * a.parts * a.splits;
-  if (items == 0) return FP2_OK;
-  cudaError_t e = fp2::launch_attention(p->dtype, D, B, a, c.plan, items, st);
+  const int64_t row_items = c.total_blocks * p->num_kv_heads * a.parts * a.splits;
+  if (row_items == 0) return FP2_OK;
+  cudaError_t e;
+  if (c.pieces > 0) {
+    e = fp2::launch_split_plan(a, c.plan, c.rows, B, c.piece_tiles, st);
+    if (e != cudaSuccess) return cuda_fail(e, "split plan kernel launch");
+  }
+  e = fp2::launch_attention(p->dtype, D, B, a, c.plan, row_items + a.adapt, st);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
   if (c.splits > 1) {
     e = fp2::launch_combine(p->dtype, D, a.o_part, a.lse_part, c.splits, static_cast<int>(c.T), p->num_q_heads, out,

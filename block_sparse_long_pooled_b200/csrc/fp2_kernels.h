@@ -69,6 +69,15 @@ struct AttnArgs {
   int num_sms;                // SMs of the device (the launch's wave width)
   float* o_part;              // [splits, T, Hq, d] f32 partial outputs (splits > 1)
   float* lse_part;            // [splits, Hq, T] f32 partial LSE (splits > 1)
+  // Adaptive splits: CTAs [0, adapt) of the launch run the pieces listed by split_plan_kernel;
+  // the rows those pieces cover are skipped by their own CTAs.  adapt = 0: none.
+  int adapt;                  // piece capacity (CTAs launched ahead of the row CTAs)
+  int32_t* row_item0;         // [rows] first piece of the row, or -1 when the row is not split
+  int2* items;                // [adapt] piece: {row, (pieces of the row << 16) | (part << 8) | piece}
+  int32_t* n_items;           // pieces planned (<= adapt)
+  int32_t* piece_cnt;         // [adapt * 2] finished pieces per (first piece of a row part, M tile)
+  float* o_slot;              // [adapt, NT * 128, d] f32 normalised partial outputs of the pieces
+  float* lse_slot;            // [adapt, NT * 128] f32 natural-log partial LSE
   uint32_t* status;
 };
 
@@ -85,6 +94,10 @@ cudaError_t launch_discover(const DiscArgs& a, const Fp2Plan& P, int64_t items, 
 cudaError_t launch_attention(int dtype, int D, int B, const AttnArgs& a, const Fp2Plan& P, int64_t items,
                              cudaStream_t stream);
 size_t attention_smem_bytes(int dtype, int D, int B);
+// Plans the adaptive pieces of one attention launch from the index's row_ptr (a.adapt > 0):
+// piece_tiles > 0 cuts rows longer than that many key tiles; 0 derives the size from the launch.
+cudaError_t launch_split_plan(const AttnArgs& a, const Fp2Plan& P, int64_t rows, int B, int piece_tiles,
+                              cudaStream_t stream);
 cudaError_t launch_combine(int dtype, int D, const float* o_part, const float* lse_part, int S, int T, int Hq,
                            void* out, float* lse, cudaStream_t stream);
 

@@ -126,10 +126,20 @@ typedef struct {
   int32_t last_n_blocks;    /* the last n query blocks of each sequence keep every key block */
   int32_t min_sparse_len;   /* sequences shorter than this keep every block */
   int32_t mean_correction;  /* nonzero: pruned blocks contribute their pooled term */
-  int32_t kv_splits;        /* count-balanced KV splits per row (paper page, Table 7): each row's key
-                               tiles are cut into this many equal ranges processed by separate CTAs
-                               and merged by their LSE; 1 = no split; 0 = automatic (split only when
-                               rows x packed parts < 296, into up to 8 ranges); at most 64 */
+  int32_t kv_splits;        /* count-balanced KV splits (paper page, Table 7): a split row's key tiles
+                               are cut into equal ranges processed by separate CTAs and merged by
+                               their LSE.
+                               >= 1: every row in this many ranges (1 = no split; at most 64);
+                               < 0:  adaptive: rows with more than -kv_splits key tiles (virtual
+                                     tiles of the mean correction + kept blocks) are cut into
+                                     ranges of at most that many tiles (at most 64 per row), the
+                                     other rows stay whole; planned on the device from the index;
+                               0:    automatic: when rows x packed parts < 296, every row in up to
+                                     8 ranges; otherwise adaptive with the range size set to the
+                                     launch's total tile work over 4 x SMs (at least 32 tiles), so
+                                     that no row outlasts a fraction of the launch's load per SM.
+                               Adaptive splits hold at most 768 ranges per fp2_attend call; rows
+                               beyond that stay whole.  Range >= -FP2_MAX_BLOCKS. */
 } fp2_sparse_params;
 
 /* Pooled block statistics (caller-owned device buffers). */
@@ -161,7 +171,8 @@ typedef struct {
   size_t qbar_bytes, kbar_bytes, vbar_bytes, kbar_mma_bytes, vbar_mma_bytes;
   size_t row_ptr_bytes, col_idx_bytes;
   size_t discover_scratch_bytes; /* the part of scratch that fp2_discover uses (status, kept bits, counts) */
-  size_t scratch_bytes;          /* scratch for fp2_pool / fp2_discover / fp2_attend (adds KV-split partials) */
+  size_t scratch_bytes;          /* scratch for fp2_pool / fp2_discover / fp2_attend (adds KV-split partials:
+                                    for adaptive splits up to 768 ranges x (128 or 256) rows x d fp32) */
   size_t prefill_scratch_bytes;  /* scratch for fp2_prefill (adds pooled and index buffers) */
 } fp2_workspace;
 

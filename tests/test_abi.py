@@ -74,6 +74,8 @@ def test_workspace_sizes():
     ({}, dict(sink_blocks=-1), fp2.FP2_ERR_INVALID_ARG),
     (dict(seqlens=(4096 * 128 + 1,)), {}, fp2.FP2_ERR_UNSUPPORTED),
     (dict(paged=True, page_size=24), {}, fp2.FP2_ERR_UNSUPPORTED),
+    ({}, dict(kv_splits=65), fp2.FP2_ERR_INVALID_ARG),
+    ({}, dict(kv_splits=-4097), fp2.FP2_ERR_INVALID_ARG),
 ])
 def test_validation_errors(kw, params, code):
     prob = _problem(**kw)
@@ -83,6 +85,27 @@ def test_validation_errors(kw, params, code):
         fp2.fp2_workspace_query(prob, fp2.make_params(**p))
     assert e.value.status == code
     assert fp2.fp2_last_error() != ""
+
+
+def test_split_modes_size_their_partials():
+    # 22 index rows x 2 parts = 44 row CTAs: few, so kv_splits = 0 splits every row uniformly into
+    # min(8, ceil(296 / 44)) = 7 ranges
+    prob = _problem()
+    one = fp2.fp2_workspace_query(prob, fp2.make_params(128, kv_splits=1))
+    auto = fp2.fp2_workspace_query(prob, fp2.make_params(128, kv_splits=0))
+    uni = fp2.fp2_workspace_query(prob, fp2.make_params(128, kv_splits=3))
+    T, Hq, d = 1333, 8, 128
+    assert uni.scratch_bytes - one.scratch_bytes >= 3 * T * Hq * d * 4
+    assert auto.scratch_bytes - one.scratch_bytes >= 7 * T * Hq * d * 4
+    # adaptive (kv_splits < 0): at most 64 ranges per row part (44 row parts here), slots of
+    # 2 x 128 packed rows x d fp32 each; many rows switch the automatic mode to adaptive as well
+    ada = fp2.fp2_workspace_query(prob, fp2.make_params(128, kv_splits=-5))
+    assert ada.scratch_bytes - one.scratch_bytes >= min(768, 44 * 64) * 256 * d * 4
+    many = _problem(seqlens=(40000,))  # 313 blocks x 2 KV heads x 2 parts: many row CTAs
+    m1 = fp2.fp2_workspace_query(many, fp2.make_params(128, kv_splits=1))
+    m0 = fp2.fp2_workspace_query(many, fp2.make_params(128, kv_splits=0))
+    assert m0.scratch_bytes - m1.scratch_bytes >= 768 * 256 * d * 4
+    assert m0.discover_scratch_bytes == m1.discover_scratch_bytes
 
 
 def test_chunked_prefill_sizes_and_rules():

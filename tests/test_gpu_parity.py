@@ -98,6 +98,41 @@ def test_kv_splits_match_oracle(case):
         assert ws.scratch_bytes > one.scratch_bytes          # partial buffers were sized: it did split
 
 
+# Adaptive splits: kv_splits < 0 cuts rows with more key tiles than -kv_splits into ranges of at
+# most that many tiles (planned on the device; the last range of a row part to finish merges them).
+# The G = 8 paged case needs more ranges than the 768 a call holds, so its later rows stay whole.
+ADAPTIVE = [
+    (small("adapt_bf16_g4", seqlens=(1500, 600), sink_blocks=2, window_blocks=4), -3),
+    (small("adapt_bf16_g8_paged", num_q_heads=16, num_kv_heads=2, seqlens=(2000, 1900), paged=True, page_size=64), -1),
+    (small("adapt_e4m3", dtype="e4m3", seqlens=(1800, 700)), -4),
+    (small("adapt_f32_d64_b64", dtype="f32", num_q_heads=4, num_kv_heads=2, head_dim=64, block_size=64,
+           seqlens=(1100,)), -5),
+    (small("adapt_bf16_g1_d64_b64", num_q_heads=2, num_kv_heads=2, head_dim=64, block_size=64,
+           seqlens=(2100, 50)), -7),
+]
+
+
+@pytest.mark.parametrize("case", ADAPTIVE, ids=lambda c: c[0].name)
+def test_adaptive_splits_match_oracle(case):
+    w, splits = case
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), kv_splits=splits)
+    Hn.compare_attention_full(run, inp, ora)
+
+
+def test_adaptive_splits_automatic_on_a_mixed_batch():
+    """kv_splits = 0 with many rows: one 16K sequence among sixty 300-token ones; its long rows
+    are cut into ranges (range size = the launch's tile work over 4 x SMs), the rest stay whole."""
+    w = small("adapt_auto_mixed", seqlens=(300,) * 60 + (16000,), sink_blocks=2, window_blocks=4)
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), kv_splits=0)
+    Hn.compare_attention_sampled(run, inp, ora, n_per_seq=16)
+
+
 def test_tiny_workload_end_to_end():
     """The 1K fp32 workload with its four planted needle blocks, through fp2_prefill."""
     import torch
