@@ -37,7 +37,7 @@ FP8_WORKLOAD = "llama8b_128k_e4m3"
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
 # taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
-ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7606532352 + 1058762752, "source_sha": "37c8408d6b14c538"}}
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7514545664 + 1065206272, "source_sha": "a9fd108a328cb068"}}
 
 
 def max_over_ranks(pg, x, device=None):
@@ -657,7 +657,8 @@ def main():
                               "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 flops x max SM clock (unit counts)",
                               "includes": "discover_kernel + scan_kernel + scatter_kernel"},
         "clocks": clocks,
-        "gpu_launches": 5 * args.steps,
+        # pool, discover (3), attention, and one of split plan (many rows) or split combine (few rows)
+        "gpu_launches": 6 * args.steps,
     }
     if not args.no_extras:
         # the same library with every block kept (alpha = 0) on the same inputs

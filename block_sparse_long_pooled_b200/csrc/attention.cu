@@ -13,9 +13,13 @@
 // correction shares the exact path's MMAs and online softmax; kept blocks and blocks >= i
 // are masked out of the virtual tiles.  The last kept block is the diagonal (causal mask).
 //
-// KV splits: with few rows, each row's key stream can be cut into `splits` contiguous ranges of
-// equal tile count (count-balanced; paper page, Table 7); every range is a separate CTA writing a
-// normalised partial O and its LSE, merged afterwards by combine_kernel.
+// KV splits (count-balanced; paper page, Table 7).  Uniform: with few rows, each row's key stream
+// is cut into `splits` contiguous ranges of equal tile count; every range is a separate CTA
+// writing a normalised partial O and its LSE, merged afterwards by combine_kernel.  Adaptive:
+// split_plan_kernel reads the index and cuts only the rows whose tile count exceeds the piece
+// size into ranges ("pieces"); CTAs [0, adapt) of the launch run the pieces (long work first),
+// the row CTAs of those rows exit at once, and the last piece of a (row, part) to finish merges
+// the pieces' partials in its epilogue.
 //
 // Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3 / 4-7  softmax for M tile 0 / 1: one TMEM lane (row) per thread; read S (and
