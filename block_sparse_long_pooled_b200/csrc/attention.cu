@@ -951,55 +951,60 @@ __global__ void __launch_bounds__(384, 1)
 // blocks), picks the piece size T (piece_tiles, or the launch's total tile work over 4 x SMs, at
 // least 32), and lists min(64, ceil(tiles / T)) pieces for every part of each row longer than T,
 // rows in index order, while they fit in a.adapt.  The pieces of one (row, part) are consecutive.
+constexpr int kPlanSmemRows = 32768;  // rows whose tile counts the plan keeps in shared memory
+
 __global__ void __launch_bounds__(1024) split_plan_kernel(const __grid_constant__ AttnArgs a,
                                                           const __grid_constant__ Fp2Plan P, int64_t rows, int BN,
                                                           int piece_tiles) {
+  extern __shared__ int32_t tiles_s[];  // [rows] when rows <= kPlanSmemRows
   __shared__ long long red[32];
   __shared__ int n_used;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t seg = (rows + 1023) / 1024;
-  const int64_t s0 = min(rows, tid * seg), s1 = min(rows, s0 + seg);
-  const int r_first = s0 < rows ? seq_of_block(P, static_cast<int>(s0 / a.Hkv)) : 0;
-  auto row_tiles = [&](int64_t x, int& rc) {
+  const bool cached = rows <= kPlanSmemRows;
+  auto row_tiles = [&](int64_t x) {
     const int b = static_cast<int>(x / a.Hkv);
-    while (rc + 1 < P.num_seqs && P.blk_off[rc + 1] <= b) ++rc;
-    const int I = P.pre_blk[rc] + (b - P.blk_off[rc]);
+    int lo = 0, hi = P.num_seqs - 1;  // the last sequence whose first block is <= b
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (P.blk_off[mid] <= b) lo = mid; else hi = mid - 1;
+    }
+    const int I = P.pre_blk[lo] + (b - P.blk_off[lo]);
     const int nk = max(0, min(a.row_ptr[x + 1] - a.row_ptr[x], I + 1));
     const int nv = (a.mean_correction && I + 1 - nk > 0) ? (I + BN - 1) / BN : 0;
     return nv + nk;
   };
-  // Block sum of one value per thread (every thread gets the total).
-  auto block_sum = [&](long long v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    long long t = 0;
-    for (int w = 0; w < 32; ++w) t += red[w];
-    __syncthreads();
-    return t;
-  };
   for (int k = tid; k < a.adapt * 2; k += 1024) a.piece_cnt[k] = 0;
   if (tid == 0) n_used = 0;
+  // Pass 1, coalesced: every row's tile count (kept in shared memory) and their sum.
+  long long loc = 0;
+  for (int64_t x = tid; x < rows; x += 1024) {
+    const int t = row_tiles(x);
+    if (cached) tiles_s[x] = t;
+    loc += t;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) loc += __shfl_xor_sync(0xFFFFFFFFu, loc, o);
+  if (lane == 0) red[warp] = loc;
+  __syncthreads();
+  long long total = 0;
+  for (int w = 0; w < 32; ++w) total += red[w];
+  __syncthreads();
   long long T = piece_tiles;
   if (T <= 0) {
-    long long loc = 0;
-    int rc = r_first;
-    for (int64_t x = s0; x < s1; ++x) loc += row_tiles(x, rc);
     const long long slots = 4LL * max(a.num_sms, 1);
-    T = max(32LL, (block_sum(loc) * a.parts + slots - 1) / slots);
+    T = max(32LL, (total * a.parts + slots - 1) / slots);
   }
   auto pieces_of = [&](int t) { return t > T ? static_cast<int>(min(64LL, (t + T - 1) / T)) : 1; };
-  // Exclusive scan of the piece counts (pieces x parts of each split row) over the rows.
-  long long loc = 0;
-  {
-    int rc = r_first;
-    for (int64_t x = s0; x < s1; ++x) {
-      const int S = pieces_of(row_tiles(x, rc));
-      if (S > 1) loc += static_cast<long long>(S) * a.parts;
-    }
+  // Pass 2: exclusive scan of the piece counts (pieces x parts of each split row) over contiguous
+  // row segments, then the piece list.
+  const int64_t seg = (rows + 1023) / 1024;
+  const int64_t s0 = min(rows, tid * seg), s1 = min(rows, s0 + seg);
+  long long cnt_loc = 0;
+  for (int64_t x = s0; x < s1; ++x) {
+    const int S = pieces_of(cached ? tiles_s[x] : row_tiles(x));
+    if (S > 1) cnt_loc += static_cast<long long>(S) * a.parts;
   }
-  long long incl = loc;
+  long long incl = cnt_loc;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -1007,13 +1012,11 @@ __global__ void __launch_bounds__(1024) split_plan_kernel(const __grid_constant_
   }
   if (lane == 31) red[warp] = incl;
   __syncthreads();
-  long long before = 0;
-  for (int w = 0; w < warp; ++w) before += red[w];
-  long long base = before + incl - loc;
-  int rc = r_first;
+  long long base = incl - cnt_loc;
+  for (int w = 0; w < warp; ++w) base += red[w];
   int used = 0;
   for (int64_t x = s0; x < s1; ++x) {
-    const int S = pieces_of(row_tiles(x, rc));
+    const int S = pieces_of(cached ? tiles_s[x] : row_tiles(x));
     const long long cnt = S > 1 ? static_cast<long long>(S) * a.parts : 0;
     if (cnt > 0 && base + cnt <= a.adapt) {
       a.row_item0[x] = static_cast<int32_t>(base);
@@ -1033,7 +1036,10 @@ __global__ void __launch_bounds__(1024) split_plan_kernel(const __grid_constant_
 
 cudaError_t launch_split_plan(const AttnArgs& a, const Fp2Plan& P, int64_t rows, int B, int piece_tiles,
                               cudaStream_t stream) {
-  split_plan_kernel<<<1, 1024, 0, stream>>>(a, P, rows, B, piece_tiles);
+  const int smem = static_cast<int>(std::min<int64_t>(rows, kPlanSmemRows) * 4);
+  const cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(split_plan_kernel), smem);
+  if (e != cudaSuccess) return e;
+  split_plan_kernel<<<1, 1024, smem, stream>>>(a, P, rows, B, piece_tiles);
   return cudaGetLastError();
 }
 

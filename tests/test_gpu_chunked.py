@@ -29,11 +29,11 @@ def _need_gpu():
     build.build()
 
 
-def chunk_case(name, seqlens_k, q_lens, **kw):
+def chunk_case(name, seqlens_k, q_lens, kv_splits=0, **kw):
     base = dict(num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=128, dtype="bf16", sink_blocks=1,
                 window_blocks=2, alpha=0.1, seed=17)
     base.update(kw)
-    return W.Workload(name=name, seqlens=tuple(seqlens_k), **base), list(q_lens)
+    return W.Workload(name=name, seqlens=tuple(seqlens_k), **base), list(q_lens), kv_splits
 
 
 CASES = [
@@ -43,6 +43,10 @@ CASES = [
     chunk_case("chunk_e4m3", (2100,), (564,), dtype="e4m3"),
     chunk_case("chunk_bf16_d64_b64", (1000,), (296,), head_dim=64, block_size=64, num_q_heads=4,
                last_n_blocks=1, sink_blocks=2, window_blocks=3),
+    # adaptive KV splits (ranges of at most 2 or 3 key tiles) over prefixes, paged, FP8
+    chunk_case("chunk_bf16_varlen_adaptive", (1280, 700, 2000), (256, 700, 720), kv_splits=-2),
+    chunk_case("chunk_e4m3_paged_adaptive", (2100, 1500), (564, 220), kv_splits=-3, dtype="e4m3", paged=True,
+               page_size=64),
 ]
 
 
@@ -99,12 +103,12 @@ def gpu_kept_chunked(rp, ci, q_lens, k_lens, B, Hkv):
 @pytest.mark.parametrize("case", CASES, ids=[c[0].name for c in CASES])
 def test_chunked_parity(case):
     from block_sparse_long_pooled_b200 import fp2
-    w, q_lens = case
+    w, q_lens, kv_splits = case
     inp = W.generate(w)
     qc, cu_q, cu_k, _ = split_queries(inp, q_lens)
     ref = oracle_chunked(inp, w, qc, cu_q, cu_k)
     prob, dev = gpu_problem(inp, w, qc, cu_q, cu_k)
-    params = Hn.gpu_params(w)
+    params = Hn.gpu_params(w, kv_splits=kv_splits)
     ws = fp2.fp2_workspace_query(prob, params)
     pst, pooled = fp2.alloc_pooled(ws, prob, "cuda")
     ist, index = fp2.alloc_index(ws, "cuda")
