@@ -37,7 +37,7 @@ FP8_WORKLOAD = "llama8b_128k_e4m3"
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
 # taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
-ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7514545664 + 1065206272, "source_sha": "a9fd108a328cb068"}}
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7531338496 + 1064892416, "source_sha": "804a18555d188493"}}
 
 
 def max_over_ranks(pg, x, device=None):
