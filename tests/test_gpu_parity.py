@@ -122,6 +122,32 @@ def test_adaptive_splits_match_oracle(case):
     Hn.compare_attention_full(run, inp, ora)
 
 
+def test_prefill_single_call_with_adaptive_splits():
+    """fp2_prefill (pool, discover and attend in one call, index and pooled buffers carved from its
+    scratch) with ranges of at most two key tiles, against the oracle, output and LSE."""
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    w = small("prefill_adaptive", seqlens=(1700, 900), sink_blocks=2, window_blocks=4)
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    dev = Hn.to_device(inp)
+    prob = Hn.make_gpu_problem(inp, dev)
+    params = Hn.gpu_params(w, kv_splits=-2)
+    ws = fp2.fp2_workspace_query(prob, params)
+    scratch = fp2.alloc_scratch(ws.prefill_scratch_bytes, "cuda")
+    out = torch.empty(inp.q.shape, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.num_q_heads, w.total_tokens), dtype=torch.float32, device="cuda")
+    fp2.fp2_prefill(prob, params, out, lse, scratch)
+    torch.cuda.synchronize()
+    assert fp2.fp2_get_device_status(scratch) == (0, 0)
+
+    class R:
+        pass
+    run = R()
+    run.out, run.lse = out, lse
+    Hn.compare_attention_full(run, inp, ora)
+
+
 def test_adaptive_splits_automatic_on_a_mixed_batch():
     """kv_splits = 0 with many rows: one 16K sequence among sixty 300-token ones; its long rows
     are cut into ranges (range size = the launch's tile work over 4 x SMs), the rest stay whole."""
