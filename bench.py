@@ -197,6 +197,18 @@ class Path:
         d, B = w.head_dim, w.block_size
         return 4.0 * d * B * B * kept + 4.0 * d * B * pruned, kept, pruned, causal
 
+    def launches_per_step(self):
+        """Kernels one step launches: pool, discover (3), attention, and with kv_splits = 0 one more
+        when the attention launch is short: the split combine (fewer than 296 row CTAs) or the
+        split plan (fewer than 16 waves of 148 SMs), following the library's automatic rule."""
+        w = self.w
+        G = w.num_q_heads // w.num_kv_heads
+        mtiles = -(-G * w.block_size // 128)
+        nt = 2 if mtiles >= 2 else 1
+        parts = -(-mtiles // nt)
+        row_ctas = self.ws.index_rows * parts
+        return 5 + (1 if row_ctas < 16 * 148 else 0)
+
     def discover_flops(self):
         """Algorithmic flops of the pooled block scores: 2 d per (q head, query block, causal key block)."""
         w = self.w
@@ -530,6 +542,10 @@ def chunked_sweep(args, dev, peaks):
             ws = fp2.fp2_workspace_query(prob, params)
             ist, ix = fp2.alloc_index(ws, dev)
             chunks.append((prob, ist, ix, s0))
+            # one scratch serves every call: size it for the largest (short chunk launches carry
+            # the adaptive-split buffers, the one-pass launch does not)
+            if ws.scratch_bytes > scratch.numel():
+                scratch = fp2.alloc_scratch(ws.scratch_bytes, dev)
 
         def run(evs=None):
             for n, (prob, ist, _, s0) in enumerate(chunks):
@@ -657,8 +673,7 @@ def main():
                               "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 flops x max SM clock (unit counts)",
                               "includes": "discover_kernel + scan_kernel + scatter_kernel"},
         "clocks": clocks,
-        # pool, discover (3), attention, and one of split plan (many rows) or split combine (few rows)
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": path.launches_per_step() * args.steps,
     }
     if not args.no_extras:
         # the same library with every block kept (alpha = 0) on the same inputs

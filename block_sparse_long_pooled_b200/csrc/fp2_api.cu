@@ -34,6 +34,10 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // plans 2-3 x SMs), and at most kMaxPieceSplits pieces per row.
 constexpr int kMaxPieces = 768;
 constexpr int kMaxPieceSplits = 64;
+// The automatic mode plans pieces only for launches of fewer row CTAs than 16 waves of a 148-SM
+// B200: longer launches balance themselves (rows grow with the query block and run heavy-first),
+// and there the plan kernel and the idle piece CTAs would cost a few percent.
+constexpr int64_t kAdaptiveRowCtas = 16 * 148;
 
 int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : (t == FP2_BF16 ? 2 : 1); }
 
@@ -185,7 +189,7 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
                                                                                    std::max<int64_t>(row_ctas, 1)));
   // Rows whose key-tile count is far above the launch's share per SM are cut into pieces planned
   // on the device (kv_splits < 0: pieces of at most -kv_splits tiles; 0 with many rows: automatic).
-  if (c.splits == 1 && s->kv_splits <= 0) {
+  if (c.splits == 1 && (s->kv_splits < 0 || (s->kv_splits == 0 && row_ctas < kAdaptiveRowCtas))) {
     c.piece_tiles = s->kv_splits < 0 ? -s->kv_splits : 0;
     c.pieces = static_cast<int>(std::min<int64_t>(kMaxPieces, row_ctas * kMaxPieceSplits));
   }

@@ -135,9 +135,10 @@ typedef struct {
                                      ranges of at most that many tiles (at most 64 per row), the
                                      other rows stay whole; planned on the device from the index;
                                0:    automatic: when rows x packed parts < 296, every row in up to
-                                     8 ranges; otherwise adaptive with the range size set to the
-                                     launch's total tile work over 4 x SMs (at least 32 tiles), so
-                                     that no row outlasts a fraction of the launch's load per SM.
+                                     8 ranges; below 2368 (16 waves of 148 SMs), adaptive with the
+                                     range size set to the launch's total tile work over 4 x SMs
+                                     (at least 32 tiles), so that no row outlasts a fraction of the
+                                     launch's load per SM; longer launches are not split.
                                Adaptive splits hold at most 768 ranges per fp2_attend call; rows
                                beyond that stay whole.  Range >= -FP2_MAX_BLOCKS. */
 } fp2_sparse_params;

@@ -101,11 +101,17 @@ def test_split_modes_size_their_partials():
     # 2 x 128 packed rows x d fp32 each; many rows switch the automatic mode to adaptive as well
     ada = fp2.fp2_workspace_query(prob, fp2.make_params(128, kv_splits=-5))
     assert ada.scratch_bytes - one.scratch_bytes >= min(768, 44 * 64) * 256 * d * 4
-    many = _problem(seqlens=(40000,))  # 313 blocks x 2 KV heads x 2 parts: many row CTAs
+    many = _problem(seqlens=(40000,))  # 313 blocks x 2 KV heads x 2 parts = 1252 row CTAs
     m1 = fp2.fp2_workspace_query(many, fp2.make_params(128, kv_splits=1))
     m0 = fp2.fp2_workspace_query(many, fp2.make_params(128, kv_splits=0))
     assert m0.scratch_bytes - m1.scratch_bytes >= 768 * 256 * d * 4
     assert m0.discover_scratch_bytes == m1.discover_scratch_bytes
+    # launches of 16 waves of 148 SMs or more are left whole in the automatic mode
+    huge = _problem(seqlens=(131072,), Hq=32, Hkv=8)  # 1024 blocks x 8 KV heads x 2 parts
+    h1 = fp2.fp2_workspace_query(huge, fp2.make_params(128, kv_splits=1))
+    h0 = fp2.fp2_workspace_query(huge, fp2.make_params(128, kv_splits=0))
+    hf = fp2.fp2_workspace_query(huge, fp2.make_params(128, kv_splits=-64))
+    assert h0.scratch_bytes == h1.scratch_bytes < hf.scratch_bytes
 
 
 def test_chunked_prefill_sizes_and_rules():

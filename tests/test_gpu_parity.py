@@ -149,8 +149,9 @@ def test_prefill_single_call_with_adaptive_splits():
 
 
 def test_adaptive_splits_automatic_on_a_mixed_batch():
-    """kv_splits = 0 with many rows: one 16K sequence among sixty 300-token ones; its long rows
-    are cut into ranges (range size = the launch's tile work over 4 x SMs), the rest stay whole."""
+    """kv_splits = 0 with many rows (1220 row CTAs, under 16 waves): one 16K sequence among sixty
+    300-token ones; its long rows are cut into ranges (range size = the launch's tile work over
+    4 x SMs), the rest stay whole."""
     w = small("adapt_auto_mixed", seqlens=(300,) * 60 + (16000,), sink_blocks=2, window_blocks=4)
     inp = W.generate(w)
     ora = Hn.oracle_discovery(inp)
