@@ -651,7 +651,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded NIAH-style generator, see DESIGN.md)",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded needle-in-a-haystack-style generator: low-rank block-persistent Q/K, planted needle key blocks and queries)",
         "config": {"workload": w.name, "seq_len": max(w.seqlens), "batch": len(w.seqlens),
                    "heads": f"{w.num_q_heads}/{w.num_kv_heads}", "head_dim": w.head_dim, "block": w.block_size,
                    "alpha": w.alpha, "sink": w.sink_blocks, "window": w.window_blocks,
