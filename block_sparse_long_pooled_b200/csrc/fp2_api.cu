@@ -512,6 +512,21 @@ fp2_status fp2_workspace_query(const fp2_problem* problem, const fp2_sparse_para
   return FP2_OK;
 }
 
+fp2_status fp2_workspace_size(const fp2_problem* problem, const fp2_sparse_params* params, size_t* pooled_bytes,
+                              size_t* index_bytes, size_t* scratch_bytes) {
+  Ctx c;
+  const fp2_status s = validate(problem, params, c);
+  if (s != FP2_OK) return s;
+  const fp2_workspace& w = c.ws;
+  if (pooled_bytes != nullptr)
+    *pooled_bytes = align_up(w.qbar_bytes) + align_up(w.kbar_bytes) + align_up(w.vbar_bytes) +
+                    align_up(w.kbar_mma_bytes) + align_up(w.vbar_mma_bytes);
+  if (index_bytes != nullptr) *index_bytes = align_up(w.row_ptr_bytes) + align_up(w.col_idx_bytes);
+  if (scratch_bytes != nullptr) *scratch_bytes = w.scratch_bytes;
+  g_last_error.clear();
+  return FP2_OK;
+}
+
 fp2_status fp2_pool(const fp2_problem* problem, const fp2_sparse_params* params, const fp2_pooled* pooled,
                     void* scratch, size_t scratch_bytes, fp2_stream_t stream) {
   Ctx c;

@@ -26,7 +26,7 @@ FP2_MAX_SEQS, FP2_MAX_BLOCKS = 128, 4096
 STATUS_NAMES = {0: "FP2_OK", 1: "FP2_ERR_INVALID_ARG", 2: "FP2_ERR_UNSUPPORTED", 3: "FP2_ERR_WORKSPACE_TOO_SMALL",
                 4: "FP2_ERR_CUDA", 5: "FP2_ERR_DEVICE_BOUNDS", 6: "FP2_ERR_TIMEOUT"}
 
-EXPORTED = ("fp2_workspace_query", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
+EXPORTED = ("fp2_workspace_query", "fp2_workspace_size", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
             "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static")
 FP2_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -97,13 +97,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P = ctypes.POINTER
     vp, sz = ctypes.c_void_p, ctypes.c_size_t
     lib.fp2_workspace_query.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_workspace)]
+    lib.fp2_workspace_size.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(sz), P(sz), P(sz)]
     lib.fp2_pool.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_pooled), vp, sz, vp]
     lib.fp2_discover.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_pooled), P(fp2_index), vp, sz, vp]
     lib.fp2_attend.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_pooled), P(fp2_index), vp, vp, vp, sz, vp]
     lib.fp2_prefill.argtypes = [P(fp2_problem), P(fp2_sparse_params), vp, vp, vp, sz, vp]
     lib.fp2_get_device_status.argtypes = [vp, P(ctypes.c_uint32)]
     lib.fp2_discover_static.argtypes = [P(fp2_problem), P(fp2_sparse_params), P(fp2_pooled), P(fp2_index), vp, vp]
-    for name in ("fp2_workspace_query", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
+    for name in ("fp2_workspace_query", "fp2_workspace_size", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
                  "fp2_get_device_status", "fp2_discover_static"):
         getattr(lib, name).restype = ctypes.c_int
     lib.fp2_last_error.argtypes = []
@@ -195,6 +196,15 @@ def fp2_workspace_query(problem: Problem, params: fp2_sparse_params) -> fp2_work
     ws = fp2_workspace()
     _check(load_library().fp2_workspace_query(ctypes.byref(problem.struct), ctypes.byref(params), ctypes.byref(ws)))
     return ws
+
+
+def fp2_workspace_size(problem: Problem, params: fp2_sparse_params) -> tuple:
+    """(pooled_bytes, index_bytes, scratch_bytes): the totals for carving the pooled buffers and the
+    index from one allocation each (256-byte aligned offsets), and the scratch size."""
+    pooled, index, scratch = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(load_library().fp2_workspace_size(ctypes.byref(problem.struct), ctypes.byref(params), ctypes.byref(pooled),
+                                             ctypes.byref(index), ctypes.byref(scratch)))
+    return pooled.value, index.value, scratch.value
 
 
 def fp2_pool(problem: Problem, params, pooled: fp2_pooled, scratch, stream=None):

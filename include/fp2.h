@@ -181,6 +181,13 @@ typedef struct {
 FP2_API fp2_status fp2_workspace_query(const fp2_problem* problem, const fp2_sparse_params* params,
                                fp2_workspace* out);
 
+/* The same validation, reporting three totals for callers that carve buffers out of single
+ * allocations: pooled_bytes holds the five fp2_pooled buffers and index_bytes row_ptr and col_idx,
+ * each buffer starting at a 256-byte aligned offset in that order; scratch_bytes is
+ * fp2_workspace.scratch_bytes.  Any output pointer may be NULL.  Host only; launches nothing. */
+FP2_API fp2_status fp2_workspace_size(const fp2_problem* problem, const fp2_sparse_params* params,
+                              size_t* pooled_bytes, size_t* index_bytes, size_t* scratch_bytes);
+
 /* Stage 1a (Figure 3, "pools block-mean statistics"): one pass over Q, K, V
  * (gathered through the page table when paged) writing every field of *pooled.
  * Clears the device status word at the start of scratch. */

@@ -1,6 +1,7 @@
 """The C ABI library without a GPU: it loads, exports what include/fp2.h declares, and its
 host-side validation and workspace sizing behave (no CUDA call is made by these paths)."""
 
+import ctypes
 import os
 import re
 import subprocess
@@ -85,6 +86,25 @@ def test_validation_errors(kw, params, code):
         fp2.fp2_workspace_query(prob, fp2.make_params(**p))
     assert e.value.status == code
     assert fp2.fp2_last_error() != ""
+
+
+def test_workspace_size_totals():
+    prob = _problem(paged=True)
+    params = fp2.make_params(128)
+    ws = fp2.fp2_workspace_query(prob, params)
+    pooled, index, scratch = fp2.fp2_workspace_size(prob, params)
+    up = lambda x: (x + 255) // 256 * 256
+    assert pooled == sum(up(b) for b in (ws.qbar_bytes, ws.kbar_bytes, ws.vbar_bytes, ws.kbar_mma_bytes,
+                                         ws.vbar_mma_bytes))
+    assert index == up(ws.row_ptr_bytes) + up(ws.col_idx_bytes)
+    assert scratch == ws.scratch_bytes
+    # every output is optional; validation is the same as fp2_workspace_query's
+    lib = fp2.load_library()
+    assert lib.fp2_workspace_size(ctypes.byref(prob.struct), ctypes.byref(params), None, None, None) == fp2.FP2_OK
+    bad = fp2.make_params(128, alpha=2.0)
+    with pytest.raises(fp2.FP2Error) as e:
+        fp2.fp2_workspace_size(prob, bad)
+    assert e.value.status == fp2.FP2_ERR_INVALID_ARG
 
 
 def test_split_modes_size_their_partials():
