@@ -33,6 +33,14 @@ METRIC = "sparse prefill attn ms + dense-equiv & achieved TFLOPS @128K BF16/FP8,
 UNIT = "TFLOP/s (dense-equivalent)"
 DEFAULT_WORKLOAD = "llama8b_128k_bf16"
 FP8_WORKLOAD = "llama8b_128k_e4m3"
+# Every configuration of the benchmark contract, measured in the default run and reported inside
+# the headline line (per_config): the tiny fp32 case, the 32K and 128K Llama-shaped layers (128K in
+# BF16 and FP8), the paged Qwen3-30B-A3B-shaped layer and the varlen paged FP8 batch; then the
+# served configuration's last-n-blocks 8 variants of the 128K BF16 and the 64K FP8 layers.
+CONFIGS = [("C1", "tiny_1k_f32"), ("C2", "llama8b_32k_bf16"), ("C3", "llama8b_128k_bf16"),
+           ("C3-fp8", "llama8b_128k_e4m3"), ("C4", "qwen30b_64k_paged_bf16"), ("C5", "varlen6_paged_e4m3"),
+           ("served-lastn8", "llama8b_128k_bf16_lastn8"), ("served-lastn8", "qwen4b_64k_e4m3_lastn8")]
+L2_BYTES = 126 * 1024 * 1024
 
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
@@ -69,6 +77,20 @@ def load_peaks():
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
                 "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def attention_peak(dtype, peaks):
+    """Dense tensor peak for the attention kernel's operand type: the measured sustained bf16 GEMM
+    rate, times the nominal ratio for e4m3 (2x, QK runs on e4m3 operands) and tf32 (1/2x, f32
+    inputs)."""
+    ratio = {"bf16": 1.0, "e4m3": 2.0, "f32": 0.5}[dtype]
+    note = {"bf16": "", "e4m3": " x2 (FP8 nominal ratio)", "f32": " x0.5 (tf32 nominal ratio)"}[dtype]
+    return peaks["bf16_tflops_sustained"] * ratio, f"{peaks['source']} bf16 sustained{note}"
+
+
+def input_bytes(w):
+    elt = {"f32": 4, "bf16": 2, "e4m3": 1}[w.dtype]
+    return w.total_tokens * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * elt
 
 
 # ------------------------------------------------------------------ clocks sampler
@@ -126,6 +148,21 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ GPU arm
 
+_INPUTS = {}
+
+
+def generate_inputs(w):
+    """Inputs of a workload, generated once and kept until another workload's are asked for (the
+    threshold parameters do not change the inputs, so the all-kept run and the oracle sample reuse
+    them)."""
+    from synth import workloads as W
+    key = (w.name, w.seqlens, w.seed, w.dtype, w.paged)
+    if key not in _INPUTS:
+        _INPUTS.clear()
+        _INPUTS[key] = W.generate(w)
+    return _INPUTS[key]
+
+
 class Path:
     """Device-resident inputs plus every buffer of the path for one workload."""
 
@@ -139,7 +176,7 @@ class Path:
         if alpha is not None:
             self.w = self.w.replace(alpha=alpha)
         w = self.w
-        inp = W.generate(w)
+        inp = generate_inputs(w)
         self.inp = inp
         self.dev = device
         self.q = inp.q.to(device)
@@ -232,8 +269,12 @@ def fp32_fma_peak_tflops(clocks):
     return 148 * 128 * 2 * mhz * 1e6 / 1e12
 
 
-def time_path(path, steps, warmup):
+def time_path(path, steps, warmup, flush=False):
+    """Device time of `steps` steps after `warmup` untimed ones (CUDA events on the launching
+    stream).  Returns (total ms, mean ms per stage).  flush: inputs fit in L2, so a 256 MB buffer is
+    written between steps and the total is the sum of the per-step (pool..attend) spans."""
     import torch
+    buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=path.q.device) if flush else None
     for _ in range(warmup):
         path.step()
     torch.cuda.synchronize()
@@ -241,6 +282,8 @@ def time_path(path, steps, warmup):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for k in range(steps):
+        if buf is not None:
+            buf.fill_(float(k))
         path.step(evs[k])
     end.record()
     torch.cuda.synchronize()
@@ -250,6 +293,8 @@ def time_path(path, steps, warmup):
         st["pool"].append(e[0].elapsed_time(e[1]))
         st["discover"].append(e[1].elapsed_time(e[2]))
         st["attend"].append(e[2].elapsed_time(e[3]))
+    if buf is not None:
+        total = sum(e[0].elapsed_time(e[3]) for e in evs)
     return total, {k: sum(v) / len(v) for k, v in st.items()}
 
 
@@ -352,7 +397,8 @@ class OracleSampler:
     longest sequence, then times exact + mean-corrected attention for n uniformly
     drawn (group, query block) pairs (all G heads, all tokens of the block).  The
     full-workload time is estimated as discovery time + mean pair time x pairs,
-    scaled by total tokens / sampled sequence tokens for varlen batches."""
+    scaled for varlen batches by the batch's dense-equivalent work over the
+    sampled sequence's (both stages grow with the square of the length)."""
 
     def __init__(self, wname):
         import numpy as np
@@ -360,7 +406,7 @@ class OracleSampler:
         from synth import workloads as W
         self.O, self.np = O, np
         self.w = w = W.WORKLOADS[wname]
-        self.inp = W.generate(w)
+        self.inp = generate_inputs(w)
         self.r = int(np.argmax(w.seqlens))
         self.p = O.SparseParams(block_size=w.block_size, alpha=w.alpha, sink_blocks=w.sink_blocks,
                                 window_blocks=w.window_blocks, last_n_blocks=w.last_n_blocks,
@@ -407,10 +453,13 @@ class OracleSampler:
                 t2 = time.perf_counter()
                 O.attend(q, k, v, kbar, vbar, counts, kept, B, scale, w.mean_correction, rows=rows)
                 t_attn += time.perf_counter() - t2
-        est = (t_disc + t_attn / max(1, n_pairs) * w.num_kv_heads * N) * (w.total_tokens / L)
+        scale_up = w.dense_equiv_flops() / w.replace(seqlens=(L,)).dense_equiv_flops()
+        est = (t_disc + t_attn / max(1, n_pairs) * w.num_kv_heads * N) * scale_up
         desc = (f"fp64 oracle: pooling + discovery of all {w.num_kv_heads} KV-head groups of the {L}-token "
                 f"sequence, attention for {n_pairs} uniformly drawn (group, query block) pairs of "
-                f"{w.num_kv_heads * N}; full time = discovery + mean pair time x pairs")
+                f"{w.num_kv_heads * N}; full time = discovery + mean pair time x pairs"
+                + (f", x{scale_up:.3f} for the batch's other sequences (dense-equivalent work ratio)"
+                   if len(w.seqlens) > 1 else ""))
         return t_disc + t_attn, est, desc
 
 
@@ -421,29 +470,52 @@ def cpu_cores():
         return os.cpu_count()
 
 
+def config_dict(w, world):
+    """The `config` object of a bench line (the same for the GPU arm and the reference arm)."""
+    ib = input_bytes(w)
+    return {"workload": w.name, "seq_len": max(w.seqlens), "batch": len(w.seqlens),
+            "heads": f"{w.num_q_heads}/{w.num_kv_heads}", "head_dim": w.head_dim, "block": w.block_size,
+            "alpha": w.alpha, "sink": w.sink_blocks, "window": w.window_blocks, "last_n": w.last_n_blocks,
+            "min_sparse_len": w.min_sparse_len, "kv": "paged (64-token pages)" if w.paged else "contiguous",
+            "parallelism": f"replicas{world}",
+            "l2": (f"inputs larger than L2 ({ib / 1e9:.2f} GB)" if ib > L2_BYTES
+                   else f"inputs fit in L2 ({ib / 1e6:.2f} MB): 256 MB written between steps")}
+
+
 def run_reference(args, rank, world):
+    """The fp64 oracle on the host cores.  It cannot run a whole 128K step in a bounded time, so each
+    step runs a bounded sample (pooling and discovery of every KV group of the longest sequence, and
+    exact + corrected attention for `pairs` whole (group, query block) pairs).  ms_per_step is that
+    sample's measured wall time; the whole-workload time is extrapolated from it
+    (extrapolated_ms_per_full_step), and value = dense-equivalent work / extrapolated time, i.e. the
+    sample's share of the work (sample_fraction = measured / extrapolated) over its measured time."""
     from synth import workloads as W
     if rank != 0:
         return
     w = W.WORKLOADS[args.workload]
     dense = w.dense_equiv_flops()
+    pairs = 32
     sampler = OracleSampler(args.workload)
     for k in range(args.warmup):
         sampler.run(2, seed=1000 + k)
     times, ests, desc = [], [], ""
     for k in range(args.steps):
-        t, est, desc = sampler.run(4, seed=k)
+        t, est, desc = sampler.run(pairs, seed=k)
         times.append(t)
         ests.append(est)
     est = statistics.mean(ests)
+    t_mean = statistics.mean(times)
     value = dense / est / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": est * 1e3, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_mean * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "seq_len": max(w.seqlens), "heads": f"{w.num_q_heads}/{w.num_kv_heads}",
-                       "head_dim": w.head_dim, "block": w.block_size, "parallelism": f"replicas{args.gpus}"},
+            "config": config_dict(w, args.gpus),
+            "extrapolated_from_pairs": pairs,
+            "extrapolated_ms_per_full_step": est * 1e3,
+            "sample_fraction": t_mean / est,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                             "sample": desc + f"; mean over {args.steps} samples of {statistics.mean(times):.1f} s"},
+                             "sample": desc + f"; each step is this sample ({t_mean:.2f} s measured, "
+                                              f"{100 * t_mean / est:.3f} % of the extrapolated full step)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -586,19 +658,78 @@ def chunked_sweep(args, dev, peaks):
     return lines
 
 
+# ------------------------------------------------------------------ per-config measurement
+
+def measure_config(wname, dev, peaks, steps, warmup, all_kept=True, cpu_pairs=0, label=None):
+    """One workload: device-timed steps (pool, discover, attend), the rooflines of the three stages,
+    the same library with every block kept, and optionally the oracle on a bounded sample."""
+    import torch
+    from synth import workloads as W
+    w = W.WORKLOADS[wname]
+    flush = input_bytes(w) <= L2_BYTES
+    path = Path(wname, dev)
+    sampler = ClockSampler(dev.index or 0)
+    sampler.start()
+    total, st = time_path(path, steps, warmup, flush=flush)
+    clocks = sampler.stop()
+    fst, bits = path.fp2.fp2_get_device_status(path.scratch)
+    if fst != path.fp2.FP2_OK:
+        raise SystemExit(f"device status {bits:#x} on {wname}")
+    ms = total / steps
+    dense = w.dense_equiv_flops()
+    ach, kept, pruned, causal = path.achieved_flops()
+    peak, peak_src = attention_peak(w.dtype, peaks)
+    attn = ach / (st["attend"] * 1e-3) / 1e12
+    pool_gbs = path.pool_bytes() / (st["pool"] * 1e-3) / 1e9
+    disc = path.discover_flops() / (st["discover"] * 1e-3) / 1e12
+    fma_peak = fp32_fma_peak_tflops(clocks)
+    e = {"label": label, "workload": wname, "dtype": w.dtype, "config": config_dict(w, 1), "steps": steps,
+         "ms_per_step": ms, "stages_ms": st, "dense_equiv_tflops": dense / (ms * 1e-3) / 1e12,
+         "achieved_tflops": ach / (ms * 1e-3) / 1e12, "sparsity": kept / causal,
+         "roofline": {"kernel": "attention_kernel", "bound": "tensor", "achieved": attn, "peak": peak,
+                      "unit": "TFLOP/s", "frac": attn / peak, "peak_source": peak_src},
+         "pool_roofline": {"bound": "hbm", "achieved": pool_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": pool_gbs / peaks["hbm_gbs"]},
+         "discover_roofline": {"bound": "alu", "achieved": disc, "peak": fma_peak, "unit": "TFLOP/s",
+                               "frac": disc / fma_peak},
+         "clocks": clocks, "launches_per_step": path.launches_per_step()}
+    del path
+    torch.cuda.empty_cache()
+    if all_kept:
+        dp = Path(wname, dev, alpha=0.0)
+        k = max(3, steps // 4)
+        dms, dst = time_path(dp, k, 2, flush=flush)
+        dach, _, _, _ = dp.achieved_flops()
+        e["all_kept"] = {"ms_per_step": dms / k, "attend_ms": dst["attend"],
+                         "attend_tflops": dach / (dst["attend"] * 1e-3) / 1e12,
+                         "attend_frac": dach / (dst["attend"] * 1e-3) / 1e12 / peak,
+                         "speedup_of_sparse": (dms / k) / ms}
+        del dp
+        torch.cuda.empty_cache()
+    if cpu_pairs > 0:
+        secs, est, desc = OracleSampler(wname).run(cpu_pairs)
+        e["cpu_baseline"] = {"value": dense / est / 1e12, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "ms_per_step_extrapolated": est * 1e3,
+                             "sample": desc + f" ({secs:.1f} s of CPU work)"}
+    return e
+
+
 # ------------------------------------------------------------------ main
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--no-extras", action="store_true", help="skip the FP8, all-kept, e2e and CPU legs")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the headline workload: skip the all-kept, e2e, CPU and per-config legs")
     ap.add_argument("--sweep", choices=["alpha", "correction", "sparsity", "chunked"], default=None,
                     help="ablation sweeps on the 64K FP8 workload instead of the benchmark line")
     args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
     if args.sweep:
         run_sweep(args.sweep, args)
         return
@@ -625,12 +756,13 @@ def main():
 
     path = Path(args.workload, dev)
     w = path.w
+    flush = input_bytes(w) <= L2_BYTES
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     sampler.start()
-    total_ms, stages = time_path(path, args.steps, args.warmup)
+    total_ms, stages = time_path(path, args.steps, args.warmup, flush=flush)
     clocks = sampler.stop()
     total_ms = max_over_ranks(pg, total_ms, dev)
     if pg:
@@ -643,8 +775,7 @@ def main():
     ach, kept, pruned, causal = path.achieved_flops()
     value = whole_job_value(dense, world, ms)
     attn_tflops = ach / (stages["attend"] * 1e-3) / 1e12
-    peak_bf16 = peaks["bf16_tflops_sustained"]
-    peak = peak_bf16 if w.dtype != "e4m3" else 2.0 * peak_bf16
+    peak, peak_src = attention_peak(w.dtype, peaks)
     sha = source_sha(os.path.join(ROOT, "block_sparse_long_pooled_b200", "csrc", "attention.cu"))
     tr = ATTN_TRAFFIC.get(w.name)
     traffic = tr["bytes"] if tr is not None and tr["source_sha"] == sha else None
@@ -652,17 +783,12 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded needle-in-a-haystack-style generator: low-rank block-persistent Q/K, planted needle key blocks and queries)",
-        "config": {"workload": w.name, "seq_len": max(w.seqlens), "batch": len(w.seqlens),
-                   "heads": f"{w.num_q_heads}/{w.num_kv_heads}", "head_dim": w.head_dim, "block": w.block_size,
-                   "alpha": w.alpha, "sink": w.sink_blocks, "window": w.window_blocks,
-                   "parallelism": f"replicas{world}",
-                   "l2": f"inputs larger than L2 ({(path.q.numel() * path.q.element_size() + 2 * path.k.numel() * path.k.element_size()) / 1e9:.2f} GB)"},
+        "config": config_dict(w, world),
         "achieved_tflops": ach / (ms * 1e-3) / 1e12,
         "sparsity": kept / causal,
         "stages_ms": stages,
         "roofline": {"kernel": "attention_kernel", "bound": "tensor", "achieved": attn_tflops, "peak": peak,
-                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": traffic,
-                     "peak_source": f"{peaks['source']} bf16 sustained" + (" x2 (FP8 nominal ratio)" if w.dtype == "e4m3" else "")},
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": traffic, "peak_source": peak_src},
         "pool_roofline": {"bound": "hbm", "achieved": path.pool_bytes() / (stages["pool"] * 1e-3) / 1e9,
                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": path.pool_bytes() / (stages["pool"] * 1e-3) / 1e9 / peaks["hbm_gbs"]},
@@ -678,7 +804,7 @@ def main():
     if not args.no_extras:
         # the same library with every block kept (alpha = 0) on the same inputs
         dense_path = Path(args.workload, dev, alpha=0.0)
-        dms, dst = time_path(dense_path, max(3, args.steps // 8), 2)
+        dms, dst = time_path(dense_path, max(3, args.steps // 8), 3, flush=flush)
         dach, _, _, _ = dense_path.achieved_flops()
         line["all_kept"] = {"ms_per_step": dms / max(3, args.steps // 8),
                             "attend_tflops": dach / (dst["attend"] * 1e-3) / 1e12,
@@ -692,19 +818,24 @@ def main():
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "mode": "pipelined: upload, fp2_prefill and download on three streams",
                        "serial_ms_per_step": serial_ms}
-        if args.workload == DEFAULT_WORKLOAD:
-            del path
-            torch.cuda.empty_cache()
-            p8 = Path(FP8_WORKLOAD, dev)
-            ms8, st8 = time_path(p8, args.steps, args.warmup)
-            a8, k8, _, c8 = p8.achieved_flops()
-            t8 = a8 / (st8["attend"] * 1e-3) / 1e12
-            line["fp8"] = {"workload": FP8_WORKLOAD, "ms_per_step": ms8 / args.steps,
-                           "value": p8.w.dense_equiv_flops() / (ms8 / args.steps * 1e-3) / 1e12,
-                           "achieved_tflops": a8 / (ms8 / args.steps * 1e-3) / 1e12, "sparsity": k8 / c8,
-                           "stages_ms": st8, "attend_tflops": t8, "attend_frac_of_fp8_peak": t8 / (2 * peak_bf16),
-                           "attend_frac_of_bf16_peak": t8 / peak_bf16}
-            del p8
+        del path
+        torch.cuda.empty_cache()
+        if args.workload == DEFAULT_WORKLOAD and world == 1:
+            per = []
+            for label, wname in CONFIGS:
+                if wname == args.workload:
+                    per.append({"label": label, "workload": wname, "same_as": "headline line"})
+                    continue
+                per.append(measure_config(wname, dev, peaks, max(5, args.steps // 2), args.warmup,
+                                          cpu_pairs=48 if rank == 0 else 0, label=label))
+            line["per_config"] = per
+            fp8 = next(e for e in per if e["workload"] == FP8_WORKLOAD)
+            line["fp8"] = {"workload": FP8_WORKLOAD, "ms_per_step": fp8["ms_per_step"],
+                           "value": fp8["dense_equiv_tflops"], "achieved_tflops": fp8["achieved_tflops"],
+                           "sparsity": fp8["sparsity"], "stages_ms": fp8["stages_ms"],
+                           "attend_tflops": fp8["roofline"]["achieved"],
+                           "attend_frac_of_fp8_peak": fp8["roofline"]["frac"],
+                           "attend_frac_of_bf16_peak": fp8["roofline"]["achieved"] / peaks["bf16_tflops_sustained"]}
         if rank == 0 and world == 1:
             secs, est, desc = OracleSampler(args.workload).run(400)
             line["cpu_baseline"] = {"value": dense / est / 1e12, "unit": UNIT, "cores": cpu_cores(),

@@ -227,8 +227,11 @@ FP2_API fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_o
  * device allocator).  The paper has no counterpart: this is fp2_discover with its scratch moved into
  * a library-owned static __device__ buffer of FP2_STATIC_SCRATCH_BYTES per GPU, held until exit.
  * Inputs (pooled) and outputs (index) are still the caller's.  Returns FP2_ERR_UNSUPPORTED when the
- * problem's fp2_workspace.discover_scratch_bytes exceeds FP2_STATIC_SCRATCH_BYTES.  Allocates nothing.  The
- * first call on a device looks up the buffer's address (make it before any stream capture).  All
+ * problem's fp2_workspace.discover_scratch_bytes exceeds FP2_STATIC_SCRATCH_BYTES.  Calls no
+ * allocator.  The first call in each CUDA context looks up the buffer's device address (cached per
+ * device with the context's id, so a new context after a device reset looks it up again); with
+ * CUDA's lazy module loading that first call is also when the driver places the buffer, so make it
+ * at start-up, before reserving the rest of device memory and before any stream capture.  All
  * calls share the buffer: calls that overlap on the GPU race, so serialise them.  status_dev
  * (device pointer, or NULL) receives a copy of the FP2_DEV_* status word of this call. */
 FP2_API fp2_status fp2_discover_static(const fp2_problem* problem, const fp2_sparse_params* params,

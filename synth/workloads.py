@@ -119,6 +119,15 @@ WORKLOADS = {
                              description="6 packed requests (cu_seqlens), GQA 4, paged FP8, min-sparse-length 8192"),
 }
 
+# The served configuration of the nestfrontier.com write-up ("A serving setup you can actually
+# test") adds last-n-blocks 8: the same layers with the last 8 query blocks of each sequence dense.
+WORKLOADS["llama8b_128k_bf16_lastn8"] = WORKLOADS["llama8b_128k_bf16"].replace(
+    name="llama8b_128k_bf16_lastn8", last_n_blocks=8,
+    description="the 128K bf16 layer with last-n-blocks 8 (the served configuration)")
+WORKLOADS["qwen4b_64k_e4m3_lastn8"] = WORKLOADS["qwen4b_64k_e4m3"].replace(
+    name="qwen4b_64k_e4m3_lastn8", last_n_blocks=8,
+    description="the Qwen3-4B-shaped 64K FP8 layer with last-n-blocks 8 (the served configuration)")
+
 
 def get_workload(name: str) -> Workload:
     return WORKLOADS[name]

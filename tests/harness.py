@@ -269,39 +269,106 @@ def check_tol(g, ref, dtype):
     return maxabs, rel
 
 
-def sample_rows(inp: W.Inputs, r: int, n: int, seed: int = 0) -> np.ndarray:
-    """(t, h) pairs of sequence r: first/last tokens, block edges, needle rows and random ones."""
-    w = inp.workload
-    L = w.seqlens[r]
-    B = w.block_size
-    rng = np.random.default_rng(1000 + seed + r)
-    toks = {0, L - 1, min(L - 1, B - 1), min(L - 1, B), L // 2}
-    toks.update(int(x) for x in rng.integers(0, L, size=n))
-    hs = rng.integers(0, w.num_q_heads, size=len(toks))
-    return np.array([[t, int(h)] for t, h in zip(sorted(toks), hs)], dtype=np.int64)
+def seq_group_kv(inp: W.Inputs, r: int, g: int):
+    """fp64 K and V of KV head g of sequence r, shaped [L, 1, d] (through the page table when paged)."""
+    import torch
+    a, b = int(inp.cu_seqlens[r]), int(inp.cu_seqlens[r + 1])
+    if inp.page_table is None:
+        return inp.dequant("k", heads=[g], tokens=slice(a, b)), inp.dequant("v", heads=[g], tokens=slice(a, b))
+    L = b - a
+    pt = inp.page_table[r:r + 1]
+    kc = inp.k_cache[:, :, g:g + 1].to(torch.float64).numpy() * inp.k_descale
+    vc = inp.v_cache[:, :, g:g + 1].to(torch.float64).numpy() * inp.v_descale
+    return O.gather_paged(kc, pt, [L]), O.gather_paged(vc, pt, [L])
 
 
-def compare_attention_sampled(run: GpuRun, inp: W.Inputs, ora: list, n_per_seq: int = 48):
+def select_pairs(inp: W.Inputs, ora: list, n_random: int = 8, seed: int = 0) -> list:
+    """Whole (sequence r, KV group g, query block i) pairs to compare at full size.
+
+    Every pair covers all G query heads of group g and every token of block i.  Chosen per
+    sequence: the first block and the last four blocks (all groups for the last two); for each
+    planted needle key block j, the query block j itself (the needle keys sit in its diagonal
+    tile) and one later block that attends to j; the four rows with the most kept blocks in the
+    oracle's index over the whole batch; every block of sequences below min_sparse_len (the
+    dense-cutoff requests) when they have at most 32 blocks, else eight of them; and n_random
+    random (group, block) pairs.  A tenth of all query rows are planted needle queries, so every
+    pair also holds needle rows.
+    """
     w = inp.workload
-    scale = 1.0 / math.sqrt(w.head_dim)
-    G = w.group
-    g_all, r_all = [], []
-    out = run.out
-    for r in range(len(w.seqlens)):
-        a, b = int(inp.cu_seqlens[r]), int(inp.cu_seqlens[r + 1])
-        if b == a:
+    rng = np.random.default_rng(4242 + seed)
+    B, Hkv = w.block_size, w.num_kv_heads
+    pairs = set()
+    heavy = []
+    for r, L in enumerate(w.seqlens):
+        if L == 0:
             continue
-        rows = sample_rows(inp, r, n_per_seq)
-        heads = sorted(set(int(h) for h in rows[:, 1]))
-        hpos = {h: x for x, h in enumerate(heads)}
-        q = inp.dequant("q", heads=heads, tokens=slice(a, b))
-        k, v = seq_kv(inp, r)
-        local = np.stack([rows[:, 0], [hpos[int(h)] for h in rows[:, 1]]], axis=1)
+        N = -(-L // B)
+        for i in (0,) + tuple(range(max(0, N - 4), N)):
+            gs = range(Hkv) if i >= N - 2 else [int(rng.integers(Hkv))]
+            for g in gs:
+                pairs.add((r, g, i))
+        for j in (inp.needle_key_blocks[r] if inp.needle_key_blocks else []):
+            if j < N:
+                pairs.add((r, int(rng.integers(Hkv)), int(j)))
+                if j + 1 < N:
+                    pairs.add((r, int(rng.integers(Hkv)), int(rng.integers(j + 1, N))))
+        if L < w.min_sparse_len:
+            blocks = range(N) if N <= 32 else sorted(rng.choice(N, size=8, replace=False))
+            for i in blocks:
+                pairs.add((r, int(rng.integers(Hkv)), int(i)))
+        for _ in range(n_random):
+            pairs.add((r, int(rng.integers(Hkv)), int(rng.integers(N))))
+        nk = ora[r].kept.sum(axis=2)            # [Hkv, N] kept blocks per row
+        for g in range(Hkv):
+            for i in range(N):
+                heavy.append((int(nk[g, i]), r, g, i))
+    heavy.sort(reverse=True)
+    for _, r, g, i in heavy[:4]:
+        pairs.add((r, g, i))
+    return sorted(pairs)
+
+
+def oracle_pairs(inp: W.Inputs, ora: list, pairs: list, kept_override: Optional[list] = None):
+    """Oracle output [n_rows, d] and LSE [n_rows] for whole (r, g, i) pairs, rows ordered pair by
+    pair, then token, then head of the group; also the matching (token, head) indices."""
+    w = inp.workload
+    B, G = w.block_size, w.group
+    scale = 1.0 / math.sqrt(w.head_dim)
+    outs, lses, toks, heads = [], [], [], []
+    by_group = {}
+    for r, g, i in pairs:
+        by_group.setdefault((r, g), []).append(i)
+    for (r, g), blocks in sorted(by_group.items()):
+        a, b = int(inp.cu_seqlens[r]), int(inp.cu_seqlens[r + 1])
+        L = b - a
+        hs = list(range(g * G, (g + 1) * G))
+        q = inp.dequant("q", heads=hs, tokens=slice(a, b))            # [L, G, d]
+        k, v = seq_group_kv(inp, r, g)                                   # [L, 1, d]
         o = ora[r]
-        Or, _ = O.attend(q, k, v, o.kbar, o.vbar, o.counts, o.kept, w.block_size, scale, w.mean_correction,
-                         rows=local, head_ids=heads, group=G)
-        idx_t = __import__("torch").from_numpy(rows[:, 0] + a).cuda()
-        idx_h = __import__("torch").from_numpy(rows[:, 1]).cuda()
-        g_all.append(out[idx_t, idx_h].float().cpu().numpy().astype(np.float64))
-        r_all.append(Or)
-    return check_tol(np.concatenate(g_all), np.concatenate(r_all), w.dtype)
+        kept = (kept_override[r] if kept_override is not None else o.kept)[g:g + 1]
+        for i in sorted(blocks):
+            t = np.arange(i * B, min(L, (i + 1) * B))
+            rows = np.stack([np.repeat(t, G), np.tile(np.arange(G), len(t))], axis=1)
+            Or, Lr = O.attend(q, k, v, o.kbar[:, g:g + 1], o.vbar[:, g:g + 1], o.counts, kept, B, scale,
+                              w.mean_correction, rows=rows, head_ids=list(range(G)), group=G)
+            outs.append(Or)
+            lses.append(Lr)
+            toks.append(rows[:, 0] + a)
+            heads.append(rows[:, 1] + g * G)
+    return np.concatenate(outs), np.concatenate(lses), np.concatenate(toks), np.concatenate(heads)
+
+
+def compare_attention_pairs(run: GpuRun, inp: W.Inputs, ref: tuple, lse: bool = True):
+    """Every element of the selected pairs' outputs (and their LSE) against the oracle's."""
+    import torch
+    O_ref, L_ref, toks, heads = ref
+    it = torch.from_numpy(toks).to(run.out.device)
+    ih = torch.from_numpy(heads).to(run.out.device)
+    g = run.out[it, ih].float().cpu().numpy().astype(np.float64)
+    maxabs, rel = check_tol(g, O_ref, inp.workload.dtype)
+    lse_err = None
+    if lse and run.lse is not None:
+        gl = run.lse[ih, it].cpu().numpy().astype(np.float64)
+        lse_err = float(np.abs(gl - L_ref).max())
+        assert lse_err < LSE_TOL[inp.workload.dtype], lse_err
+    return {"rows": int(len(toks)), "max_abs": maxabs, "rel_l2": rel, "lse_max_abs": lse_err}

@@ -5,7 +5,8 @@ tails, every supported (dtype, head_dim, block) kernel, GQA groups 1/2/4/8,
 contiguous and paged K/V (page sizes 16/64/128), varlen batches with a dense
 cutoff, alpha = 0, last-n rows, mean correction off, an external index, and
 device-side bounds checks.  The five workloads at full size compare the whole
-block index and sampled output rows.
+block index and every element of selected whole (KV group, query block) pairs
+of the output and the LSE.
 """
 
 import math
@@ -157,7 +158,8 @@ def test_adaptive_splits_automatic_on_a_mixed_batch():
     ora = Hn.oracle_discovery(inp)
     rp, ci = Hn.oracle_csr(ora)
     run = Hn.run_gpu(inp, external_index=(rp, ci), kv_splits=0)
-    Hn.compare_attention_sampled(run, inp, ora, n_per_seq=16)
+    pairs = Hn.select_pairs(inp, ora, n_random=1)
+    Hn.compare_attention_pairs(run, inp, Hn.oracle_pairs(inp, ora, pairs))
 
 
 def test_tiny_workload_end_to_end():
@@ -193,18 +195,37 @@ FULL = ["llama8b_32k_bf16", "llama8b_128k_bf16", "llama8b_128k_e4m3", "qwen30b_6
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_workloads(name):
+    """A full-size workload: the pooled means, the whole index, and whole (KV group, query block)
+    pairs of the output and LSE (every head of the group, every token of the block; needle blocks,
+    the last blocks, the heaviest rows and the dense-cutoff requests among them), first attending on
+    the oracle's index, then, when no borderline block differs, on the library's own index."""
+    import torch
     w = W.WORKLOADS[name]
     inp = W.generate(w)
     ora = Hn.oracle_discovery(inp)
     rp, ci = Hn.oracle_csr(ora)
-    run = Hn.run_gpu(inp, external_index=(rp, ci), lse=False)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), lse=True)
     Hn.compare_pooled(run, inp, ora)
     stats = Hn.compare_index(run, inp, ora)
+    pairs = Hn.select_pairs(inp, ora)
+    assert len(pairs) >= 32
+    ref = Hn.oracle_pairs(inp, ora, pairs)
+    r1 = Hn.compare_attention_pairs(run, inp, ref)
     print(f"{name}: density {stats['density']*100:.2f}%  borderline {stats['borderline_blocks']} "
-          f"mismatched {stats['borderline_mismatches']}")
-    Hn.compare_attention_sampled(run, inp, ora)
+          f"mismatched {stats['borderline_mismatches']}  pairs {len(pairs)} rows {r1['rows']} "
+          f"max-abs {r1['max_abs']:.2e} rel-L2 {r1['rel_l2']:.2e} lse {r1['lse_max_abs']:.2e}")
     if name == "llama8b_128k_bf16":
         assert 0.04 <= stats["density"] <= 0.06
+    if w.min_sparse_len > 0:
+        dense_pairs = [p for p in pairs if w.seqlens[p[0]] < w.min_sparse_len]
+        assert len(dense_pairs) >= 2 * w.num_kv_heads
+    del run
+    torch.cuda.empty_cache()
+    if stats["borderline_mismatches"] == 0:
+        run2 = Hn.run_gpu(inp, lse=True)
+        r2 = Hn.compare_attention_pairs(run2, inp, ref)
+        print(f"{name} (own index): max-abs {r2['max_abs']:.2e} rel-L2 {r2['rel_l2']:.2e} "
+              f"lse {r2['lse_max_abs']:.2e}")
 
 
 # More than 1024 key blocks: 32 score rows of a tile no longer fit in shared memory, so discovery
@@ -225,12 +246,12 @@ def test_long_sequences_smaller_discovery_tiles(w):
     inp = W.generate(w)
     ora = Hn.oracle_discovery(inp, head_chunk=4)
     rp, ci = Hn.oracle_csr(ora)
-    run = Hn.run_gpu(inp, external_index=(rp, ci), lse=False)
+    run = Hn.run_gpu(inp, external_index=(rp, ci), lse=True)
     Hn.compare_pooled(run, inp, ora)
     stats = Hn.compare_index(run, inp, ora)
     print(f"{w.name}: density {stats['density']*100:.2f}%  borderline {stats['borderline_blocks']} "
           f"mismatched {stats['borderline_mismatches']}")
-    Hn.compare_attention_sampled(run, inp, ora, n_per_seq=32)
+    Hn.compare_attention_pairs(run, inp, Hn.oracle_pairs(inp, ora, Hn.select_pairs(inp, ora)))
 
 
 def test_page_table_out_of_range_is_reported_not_faulted():

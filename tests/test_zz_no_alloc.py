@@ -83,3 +83,36 @@ def test_static_discovery_rejects_oversized_problem():
     with pytest.raises(fp2.FP2Error) as e:
         fp2.fp2_discover_static(prob, params, pst, ix)
     assert e.value.status == fp2.FP2_ERR_UNSUPPORTED and "static buffer" in str(e.value)
+
+
+def test_static_discovery_reports_device_status_to_caller():
+    """A device-side condition seen during the call (here: more kept blocks than col_capacity)
+    reaches the caller's status_dev word.  scan_kernel raises FP2_DEV_CAPACITY and scatter_kernel
+    writes no row that would end past the capacity, so nothing is written out of bounds."""
+    import torch
+    from block_sparse_long_pooled_b200 import fp2
+    from tests import harness as Hn
+    w = W.Workload(name="noalloc_cap", seqlens=(1200,), num_q_heads=8, num_kv_heads=2, head_dim=128,
+                   block_size=128, dtype="bf16", sink_blocks=1, window_blocks=2, alpha=0.1, seed=13)
+    inp = W.generate(w)
+    dev = Hn.to_device(inp)
+    prob = Hn.make_gpu_problem(inp, dev)
+    params = Hn.gpu_params(w)
+    ws = fp2.fp2_workspace_query(prob, params)
+    pst, _ = fp2.alloc_pooled(ws, prob, "cuda")
+    scratch = fp2.alloc_scratch(ws.scratch_bytes, "cuda")
+    fp2.fp2_pool(prob, params, pst, scratch)
+    rp = torch.zeros(ws.index_rows + 1, dtype=torch.int32, device="cuda")
+    ci = torch.full((4,), -7, dtype=torch.int32, device="cuda")
+    ix = fp2.fp2_index(rp.data_ptr(), ci.data_ptr(), 1)       # room for one column only
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    fp2.fp2_discover_static(prob, params, pst, ix, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & fp2.FP2_DEV_CAPACITY
+    assert int(rp[-1].item()) > 1                               # the true count is still reported
+    assert torch.all(ci[1:] == -7)                              # nothing written past the capacity
+    # a clean call afterwards starts from a cleared status word
+    ref_st, ref = fp2.alloc_index(ws, "cuda")
+    fp2.fp2_discover_static(prob, params, pst, ref_st, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
