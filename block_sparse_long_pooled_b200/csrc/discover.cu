@@ -3,13 +3,31 @@
 // blocks, per KV head"; backend flags of the nestfrontier.com write-up: sink, window,
 // last-n-blocks, min sparse q len).
 //
-// discover_kernel: one CTA (16 warps) per (sequence, tile of TI query blocks, KV head).  The G
-//   pooled queries of every query block in the tile (up to 32 rows) and stages of 256 pooled
-//   keys x 16 dimensions are staged in shared memory (cp.async, a ring of three buffers); the
-//   scores are a small fp32 GEMM in which each thread owns 8 rows x 2 keys and each warp 8 rows
-//   x 64 keys.  All scores of the tile stay in shared memory, so the row max and the threshold
-//   test need no second pass.  Output: one bit per causal (row, key block) plus a kept count
-//   per row.
+// discover_kernel: one CTA per (sequence, tile of TI = 128 / G query blocks, KV head).  Its 128
+//   score rows are the (query block, head) pairs of the tile (row m = query block m / G, head
+//   m % G of the group) and form the M = 128 operand of tcgen05 MMAs; pooled keys stream in chunks
+//   of 128 key blocks (N = 128) and the scores of a chunk land in tensor memory, one row per TMEM
+//   lane.  The pooled means are fp32; the decision to keep a block must match an fp64 evaluation
+//   outside a 1e-3 band, so each operand x is split into two bf16 planes, hi = bf16(x) and
+//   lo = bf16(x - hi), and a score is hi.hi + hi.lo + lo.hi (three bf16 MMAs accumulating in
+//   fp32): the dropped lo.lo term and the rounding of lo are both ~2^-16 of |x|, far inside the
+//   band.  The rows need their maximum over every causal key block before any block can be
+//   tested, so the chunks run twice: pass 1 takes the row maxima, pass 2 recomputes the scores
+//   (the tensor cores are cheap next to everything else here) and tests them against
+//   max + ln alpha.  Warp roles (416 threads):
+//     warps 0-3   epilogue: one TMEM lane quarter each, so thread t owns score row t; reads a
+//                 chunk's 128 scores, releases the TMEM buffer, pass 1 updates the row max, pass
+//                 2 builds 4 words of kept bits that are OR-ed over the G heads of each query
+//                 block in shared memory (GQA union), and writes the words (with the forced
+//                 blocks: sink, window/diagonal, last-n rows) and the per-row counts.
+//     warps 4-11  converters: load fp32 pooled rows (coalesced 16-byte loads, 16 in flight per
+//                 thread), split them into the hi/lo bf16 planes and store them in the
+//                 128-byte-swizzled K-major layout the MMA reads: the query tile once, then
+//                 every key chunk of both passes into a ring of NST stages.
+//     warp 12     MMA issuer: 3 x D/16 MMAs per chunk into one of four 128-column TMEM buffers.
+//   Every wait is an mbarrier wait with a time limit; after a timeout every role runs its loop to
+//   the end without work, so the index written is still consistent (forced blocks only) and the
+//   status word says FP2_DEV_TIMEOUT.
 // scan_kernel: exclusive scan of the row counts into row_ptr (one CTA).
 // scatter_kernel: one warp per row turns its bit words into ascending column ids.
 #include <math_constants.h>
@@ -19,32 +37,83 @@
 
 namespace fp2 {
 
-constexpr int kThreads = 512;  // 16 warps
-constexpr int kWarps = kThreads / 32;
-constexpr int kKC = 256;       // key blocks per staged chunk (4 key groups x 64)
-constexpr int kDS = 16;        // head dimensions per stage
-constexpr int kKS = kDS + 4;   // padded stage row (conflict-free 16-byte reads)
-constexpr int kNB = 3;         // stage buffers: two stages in flight while one is used
-constexpr int kRows = 32;      // score rows a CTA computes (TI * G <= 32; the rest are zero)
+template <int D>
+struct DiscCfg {
+  static constexpr int ROWS = 128;                 // M: score rows of a CTA
+  static constexpr int KEYS = 128;                 // N: key blocks per chunk
+  static constexpr int UPR = D / 8;                // 8-element units per pooled row
+  static constexpr int PLANE = 128 * D * 2;        // one bf16 plane of 128 rows (query tile or key chunk)
+  static constexpr int NST = D == 64 ? 4 : 2;      // key-chunk stages (hi + lo planes each)
+  static constexpr int NBUF = 4;                   // 128-column score buffers in TMEM
+  static constexpr int NCONV = 8;                  // converter warps
+  static constexpr int THREADS = (4 + NCONV + 1) * 32;
+  static constexpr int OFF_AHI = 0, OFF_ALO = PLANE, OFF_B = 2 * PLANE;
+  static constexpr int OFF_BAR = OFF_B + NST * 2 * PLANE;
+  static constexpr int NBAR = 1 + 2 * NST + 2 * NBUF + 1;
+  static constexpr int OFF_UNION = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;  // [2][128][4] u32
+  static constexpr int OFF_CNT = OFF_UNION + 2 * 128 * 4 * 4;            // [128] int
+  static constexpr int OFF_MISC = OFF_CNT + 128 * 4;                     // TMEM address, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;                // + 1024-byte alignment slack
+  // bf16 x bf16 -> f32, both operands K-major, M = 128, N = 128.
+  static constexpr uint32_t IDESC = make_idesc(1u, 1u, 0u, 0u, 128u, 128u);
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+  static_assert(OFF_BAR % 8 == 0 && OFF_UNION % 16 == 0, "shared-memory alignment");
+  static_assert((128 * UPR) % (NCONV * 32) == 0, "converter work split");
+};
 
-FP2_DEVICE void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+// 64 consecutive TMEM columns of this thread's lane, with the wait in the same statement so that
+// no use of the registers is scheduled before the data has landed.
+FP2_DEVICE void tmem_ld_row64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr + 0u), "r"(taddr + 32u)
+      : "memory");
 }
-// 16-byte shared-memory load kept where it is written (volatile: not sunk towards its use).
-FP2_DEVICE float4 lds128(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
+
+// Bounded wait used only to drain the MMAs in flight before TMEM is freed (ignores the abort flag).
+FP2_DEVICE void drain_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) {
+      set_status(status, FP2_DEV_TIMEOUT);
+      return;
+    }
+  }
 }
-FP2_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-FP2_DEVICE void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+
+FP2_DEVICE void epilogue_bar_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Bits of word w (blocks 32w .. 32w+31) that lie in [lo, hi].
+FP2_DEVICE uint32_t range_bits(int lo, int hi, int w) {
+  const int base = 32 * w;
+  const int a = max(lo, base), b = min(hi, base + 31);
+  if (a > b) return 0u;
+  const int len = b - a + 1;
+  return (len == 32 ? 0xFFFFFFFFu : ((1u << len) - 1u)) << (a - base);
+}
+
+// Split 8 fp32 values into the 16-byte hi and lo bf16 units: hi = bf16(x), lo = bf16(x - hi).
+FP2_DEVICE void split_bf16x8(const float4& a, const float4& b, uint4& hi, uint4& lo) {
+  const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    h[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+    const float r0 = x[2 * e] - __uint_as_float(h[e] << 16);
+    const float r1 = x[2 * e + 1] - __uint_as_float(h[e] & 0xFFFF0000u);
+    l[e] = pack_bf16x2(r0, r1);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) discover_kernel(const DiscArgs a, const Fp2Plan P) {
-  extern __shared__ __align__(16) float smem[];
+__global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const __grid_constant__ DiscArgs a,
+                                                                         const __grid_constant__ Fp2Plan P) {
+  using C = DiscCfg<D>;
   int r, it, g;
   if (!map_heavy_first(P, a.TI, a.Hkv, blockIdx.x, r, it, g)) return;
   // Query block i of the sequence (or chunk) is absolute key block I = pre + i.
@@ -55,10 +124,9 @@ __global__ void __launch_bounds__(kThreads) discover_kernel(const DiscArgs a, co
   const int bo = P.blk_off[r], kbo = P.k_blk_off[r];
   const int J1 = pre + i1;  // key blocks [0, J1) are visible to some row of the tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const bool dense = a.dense_all || L < a.min_sparse_len;
 
-  if (dense) {  // every causal block kept
-    for (int ii = warp; ii < nI; ii += kWarps) {
+  if (a.dense_all || L < a.min_sparse_len) {  // every causal block kept
+    for (int ii = warp; ii < nI; ii += C::THREADS / 32) {
       const int i = i0 + ii, I = pre + i;
       const int64_t row = static_cast<int64_t>(bo + i) * a.Hkv + g;
       const int nw = (I + 32) / 32;
@@ -71,162 +139,217 @@ __global__ void __launch_bounds__(kThreads) discover_kernel(const DiscArgs a, co
     return;
   }
 
-  constexpr int QS = D + 4;  // padded pooled-query row
-  constexpr int NH = D / kDS;  // stages per key chunk
-  const int SPP = a.SP + 8;    // score row stride
-  float* qs = smem;                    // [kRows][QS]
-  float* ks = qs + kRows * QS;         // [kNB][kKC][kKS]: stage being used, two in flight
-  float* sc = ks + kNB * kKC * kKS;    // [TI*G][SPP]
-  float* thr = sc + a.TI * G * SPP;    // [32]
-  int* cnt = reinterpret_cast<int*>(thr + 32);  // [32] kept blocks per query block
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* a_full = bars;
+  uint64_t* b_full = a_full + 1;
+  uint64_t* b_empty = b_full + C::NST;
+  uint64_t* s_full = b_empty + C::NST;
+  uint64_t* s_empty = s_full + C::NBUF;
+  uint64_t* mma_done = s_empty + C::NBUF;
+  uint32_t* ubuf = reinterpret_cast<uint32_t*>(smem + C::OFF_UNION);  // [2][128][4]
+  int* cnt = reinterpret_cast<int*>(smem + C::OFF_CNT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
-  for (int idx = tid; idx < kRows * (D / 4); idx += kThreads) {
-    const int row = idx / (D / 4), c4 = idx % (D / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (row < rows) {
-      const int ii = row / G, hl = row % G;
-      v = reinterpret_cast<const float4*>(a.qbar)[(static_cast<int64_t>(bo + i0 + ii) * a.Hq + g * G + hl) * (D / 4) + c4];
-    }
-    *reinterpret_cast<float4*>(&qs[row * QS + c4 * 4]) = v;
+  const int nch = (J1 + C::KEYS - 1) / C::KEYS;
+  const int nq = 2 * nch;  // pass 1 then pass 2 over the same chunks
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
   }
-  if (tid < 32) cnt[tid] = 0;
-
-  // Stage st covers key blocks [c*kKC, c*kKC + kKC) and dimensions [h*kDS, h*kDS + kDS) with
-  // c = st / NH, h = st % NH; a ring of kNB buffers keeps stages st+1 and st+2 streaming in
-  // while stage st is used (an L2 round trip is longer than one stage's arithmetic).
-  // Each thread copies the same two 16-byte pieces of every stage: key rows jl and jl + 128 of
-  // the chunk, dimensions [4*c4, 4*c4 + 4) of the stage.
-  const int nst = (J1 + kKC - 1) / kKC * NH;
-  const int jl = tid >> 2, c4l = tid & 3;
-  const int64_t key_stride = static_cast<int64_t>(a.Hkv) * D;
-  const float* kbase = a.kbar + (static_cast<int64_t>(kbo + jl) * a.Hkv + g) * D + c4l * 4;
-  auto load_stage = [&](int st, int buf) {
-    const int j0 = (st / NH) * kKC, d0 = (st % NH) * kDS;
-    float* dst = ks + buf * (kKC * kKS) + jl * kKS + c4l * 4;
-    const float* src = kbase + j0 * key_stride + d0;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (j0 + jl + 128 * q < J1)
-        cp_async16(dst + 128 * q * kKS, src + 128 * q * key_stride);
-      else
-        *reinterpret_cast<float4*>(dst + 128 * q * kKS) = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid == 32) {
+    mbar_init(a_full, C::NCONV);
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(&b_full[s], C::NCONV);
+      mbar_init(&b_empty[s], 1);
     }
-    cp_async_commit();
-  };
-  // Thread tile: rows 8 * (warp & 3) + n (n < 8) and keys 64 * (warp >> 2) + lane + 32m (m < 2)
-  // of the chunk.  The query loads of a warp are pure broadcasts (one address) and its key
-  // loads read 32 distinct rows, so every shared-memory wavefront carries 128 useful bytes.
-  const int r0 = 8 * (warp & 3);
-  const int kb0 = 64 * (warp >> 2) + lane;
-  float acc[8][2];
-#pragma unroll
-  for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = 0.f;
+    for (int b = 0; b < C::NBUF; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int x = tid; x < 2 * 128 * 4; x += C::THREADS) ubuf[x] = 0u;
+  for (int x = tid; x < 128; x += C::THREADS) cnt[x] = 0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  load_stage(0, 0);
-  if (nst > 1) load_stage(1, 1);
-  for (int st = 0; st < nst; ++st) {
-    if (st + 1 < nst)
-      cp_async_wait<1>();  // stage st has landed; stage st+1 may still be in flight
-    else
-      cp_async_wait<0>();
-    // Stage st (and, on the first pass, the query rows) is visible to all; every thread is
-    // done with stage st-1, whose buffer the next load refills.
-    __syncthreads();
-    if (st + 2 < nst) load_stage(st + 2, (st + 2) % kNB);
-    const int h = st % NH, j0 = (st / NH) * kKC;
-    if (j0 + 64 * (warp >> 2) < J1 && r0 < rows) {  // warps with no visible key or no row idle
-      const uint32_t kp = smem_u32(ks + (st % kNB) * (kKC * kKS) + kb0 * kKS);
-      const uint32_t qp = smem_u32(qs + r0 * QS + h * kDS);
-      // Software pipeline: the operands of step k+1 are requested before the FMAs of step k, so
-      // each warp's shared-memory loads overlap its own arithmetic (the warps of a CTA run in
-      // lock step between barriers, so overlap across warps cannot be relied on).
-      float4 qv[2][8], kv[2][2];
-      auto load_step = [&](int k, int b) {
+  if (warp >= 4 && warp < 4 + C::NCONV) {
+    // ------------------------------------------------------------------ converters
+    // Thread ct owns the 8-element unit `col8` of rows r0, r0 + RSTEP, ...; unit col8 holds d
+    // 8*col8 .. +7, which is 128-byte chunk col8 / 8, 16-byte unit col8 % 8 of the swizzled row.
+    constexpr int RSTEP = C::NCONV * 32 / C::UPR;
+    constexpr int NU = 128 / RSTEP;
+    const int ct = tid - 128;
+    const int col8 = ct % C::UPR, r0 = ct / C::UPR;
+    const int chunk_off = (col8 >> 3) * (128 * 128);
+    auto convert = [&](uint8_t* hi_base, uint8_t* lo_base, auto src_of) {
+      float4 x[NU][2];
 #pragma unroll
-        for (int n = 0; n < 8; ++n) qv[b][n] = lds128(qp + 4u * (n * QS + k));
-#pragma unroll
-        for (int m = 0; m < 2; ++m) kv[b][m] = lds128(kp + 4u * (32 * m * kKS + k));
-      };
-      load_step(0, 0);
-#pragma unroll
-      for (int k = 0; k < kDS; k += 4) {
-        const int b = (k >> 2) & 1;
-        if (k + 4 < kDS) load_step(k + 4, b ^ 1);
-        // Dimension by dimension over all 16 accumulators: consecutive FMAs are independent.
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-          for (int m = 0; m < 2; ++m) acc[n][m] = fmaf(qv[b][n].x, kv[b][m].x, acc[n][m]);
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-          for (int m = 0; m < 2; ++m) acc[n][m] = fmaf(qv[b][n].y, kv[b][m].y, acc[n][m]);
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-          for (int m = 0; m < 2; ++m) acc[n][m] = fmaf(qv[b][n].z, kv[b][m].z, acc[n][m]);
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-#pragma unroll
-          for (int m = 0; m < 2; ++m) acc[n][m] = fmaf(qv[b][n].w, kv[b][m].w, acc[n][m]);
+      for (int k = 0; k < NU; ++k) {
+        const float* p = src_of(r0 + RSTEP * k);
+        if (p != nullptr) {
+          x[k][0] = __ldg(reinterpret_cast<const float4*>(p + 8 * col8));
+          x[k][1] = __ldg(reinterpret_cast<const float4*>(p + 8 * col8 + 4));
+        } else {
+          x[k][0] = x[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
-      if (h == NH - 1) {  // the chunk's dot products are complete
 #pragma unroll
-        for (int n = 0; n < 8; ++n)
+      for (int k = 0; k < NU; ++k) {
+        const int row = r0 + RSTEP * k;
+        uint4 hi, lo;
+        split_bf16x8(x[k][0], x[k][1], hi, lo);
+        const int off = chunk_off + row * 128 + (((col8 & 7) ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(hi_base + off) = hi;
+        *reinterpret_cast<uint4*>(lo_base + off) = lo;
+      }
+      fence_proxy_async_smem();  // the tensor core reads the planes through the async proxy
+      __syncwarp();
+    };
+    const int64_t qrow0 = static_cast<int64_t>(bo + i0) * a.Hq + static_cast<int64_t>(g) * G;
+    convert(smem + C::OFF_AHI, smem + C::OFF_ALO, [&](int m) -> const float* {
+      if (m >= rows) return nullptr;
+      return a.qbar + (qrow0 + static_cast<int64_t>(m / G) * a.Hq + (m % G)) * D;
+    });
+    if (lane == 0) mbar_arrive(a_full);
+    for (int q = 0; q < nq; ++q) {
+      const int stage = q % C::NST, use = q / C::NST;
+      if (use > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&b_empty[stage], (use - 1) & 1, abort_flag, a.status)))
+        break;
+      const int j0 = (q % nch) * C::KEYS;
+      uint8_t* hb = smem + C::OFF_B + stage * 2 * C::PLANE;
+      convert(hb, hb + C::PLANE, [&](int n) -> const float* {
+        const int j = j0 + n;
+        if (j >= J1) return nullptr;
+        return a.kbar + (static_cast<int64_t>(kbo + j) * a.Hkv + g) * D;
+      });
+      if (lane == 0) mbar_arrive(&b_full[stage]);
+    }
+  } else if (warp == 4 + C::NCONV) {
+    // ------------------------------------------------------------------ MMA issuer
+    bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(a_full, 0, abort_flag, a.status));
+    for (int q = 0; q < nq && ok; ++q) {
+      const int stage = q % C::NST, buf = q % C::NBUF;
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(&b_full[stage], (q / C::NST) & 1, abort_flag, a.status));
+      if (ok && q >= C::NBUF)
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_empty[buf], ((q / C::NBUF) - 1) & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t dcol = tmem + buf * C::KEYS;
+      const uint32_t bbase = sbase + C::OFF_B + stage * 2 * C::PLANE;
 #pragma unroll
-          for (int m = 0; m < 2; ++m) {
-            const int row = r0 + n, j = j0 + kb0 + 32 * m;
-            if (row < rows && j < J1) sc[row * SPP + j] = acc[n][m] * a.scale;
-            acc[n][m] = 0.f;
+      for (int t = 0; t < 3; ++t) {  // hi.hi, hi.lo, lo.hi
+        const uint64_t ad0 = smem_desc_sw128(sbase + (t == 2 ? C::OFF_ALO : C::OFF_AHI), 16, 1024);
+        const uint64_t bd0 = smem_desc_sw128(bbase + (t == 1 ? C::PLANE : 0), 16, 1024);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = static_cast<uint32_t>((k >> 2) * (128 * 128) + (k & 3) * 32);
+          umma_ss_warp<1>(dcol, ad0 + (off >> 4), bd0 + (off >> 4), C::IDESC, (t > 0 || k > 0) ? 1u : 0u);
+        }
+      }
+      umma_commit_warp(&b_empty[stage]);
+      umma_commit_warp(&s_full[buf]);
+    }
+    umma_commit_warp(mma_done);
+    if (lane == 0) drain_wait(mma_done, 0, a.status);
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------------ epilogue
+    const int m = warp * 32 + lane;  // score row = TMEM lane
+    const bool valid = m < rows;
+    const int ii = valid ? m / G : 0;
+    const int I = pre + i0 + ii;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const float scale = a.scale;
+    const int win = max(a.window, 1);
+    float mrun = -CUDART_INF_F, thr = CUDART_INF_F;
+    bool ok = true;
+    for (int q = 0; q < nq; ++q) {
+      const int buf = q % C::NBUF, c = q % nch, j0 = c * C::KEYS;
+      const bool pass2 = q >= nch;
+      if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (q / C::NBUF) & 1, abort_flag, a.status));
+      if (ok) tc_fence_after();
+      if (pass2 && q == nch) thr = mrun + a.ln_alpha;
+      const int lim = I - j0;  // columns e <= lim are causal for this row
+      // The chunk's 128 scores in two halves of 64 columns (fewer live registers).
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t v[64];
+        if (ok) tmem_ld_row64(tmem + lane_base + buf * C::KEYS + hf * 64, v);
+        if (hf == 1) {  // the buffer has been read: hand it back to the MMA warp
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_empty[buf]);
+        }
+        if (!ok || !valid) continue;
+        const int lh = lim - hf * 64;  // causal limit within this half
+        if (!pass2) {
+          if (lh >= 63) {
+            float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+            for (int e = 0; e < 64; e += 8)
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                m4[u] = fmax3(m4[u], __uint_as_float(v[e + 2 * u]) * scale, __uint_as_float(v[e + 2 * u + 1]) * scale);
+            mrun = fmax3(mrun, fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              if (e <= lh) mrun = fmaxf(mrun, __uint_as_float(v[e]) * scale);
           }
+        } else {
+#pragma unroll
+          for (int wh = 0; wh < 2; ++wh) {
+            uint32_t bits = 0u;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int col = 32 * wh + e;
+              const bool keep = (__uint_as_float(v[col]) * scale >= thr) && (col <= lh);
+              bits |= static_cast<uint32_t>(keep) << e;
+            }
+            if (bits != 0u) atomicOr(&ubuf[((c & 1) * 128 + ii) * 4 + 2 * hf + wh], bits);
+          }
+        }
+      }
+      if (pass2) {
+        epilogue_bar_sync();
+        // Union over the heads of each query block is complete: add the forced blocks and write.
+        for (int x = m; x < a.TI * 4; x += 128) {
+          const int iw = x >> 2, wq = x & 3;
+          const int i = i0 + iw;
+          uint32_t* slot = &ubuf[((c & 1) * 128 + iw) * 4 + wq];
+          if (i < i1) {
+            const int Iw = pre + i, w = 4 * c + wq;
+            if (w <= (Iw >> 5)) {
+              uint32_t word = *slot;
+              word |= range_bits(0, a.sink - 1, w) | range_bits(Iw - win + 1, Iw, w);
+              if (i >= N - a.last_n) word = 0xFFFFFFFFu;
+              word &= range_bits(0, Iw, w);
+              a.bitmask[(static_cast<int64_t>(bo + i) * a.Hkv + g) * a.W + w] = word;
+              if (word != 0u) atomicAdd(&cnt[iw], __popc(word));
+            }
+          }
+          *slot = 0u;
+        }
       }
     }
+    epilogue_bar_sync();
+    for (int x = m; x < nI; x += 128) a.counts[static_cast<int64_t>(bo + i0 + x) * a.Hkv + g] = cnt[x];
   }
-  __syncthreads();
 
-  // Row max over every causal key block (forced ones included), then the threshold.  Four
-  // independent running maxima per lane.
-  for (int row = warp; row < rows; row += kWarps) {
-    const int I = pre + i0 + row / G;
-    const float* sr = sc + row * SPP;
-    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, m2 = -CUDART_INF_F, m3 = -CUDART_INF_F;
-    int j = lane;
-    for (; j + 96 <= I; j += 128) {
-      m0 = fmaxf(m0, sr[j]);
-      m1 = fmaxf(m1, sr[j + 32]);
-      m2 = fmaxf(m2, sr[j + 64]);
-      m3 = fmaxf(m3, sr[j + 96]);
-    }
-    for (; j <= I; j += 32) m0 = fmaxf(m0, sr[j]);
-    float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (lane == 0) thr[row] = m + a.ln_alpha;
-  }
+  tc_fence_before();
   __syncthreads();
-
-  // One warp per (query block, 32-block word): forced blocks, or any head of the group at or
-  // above its threshold.
-  const int win = max(a.window, 1);
-  const int wmax = (J1 - 1 + 32) / 32;  // words of the tile's last query block
-  for (int p = warp; p < nI * wmax; p += kWarps) {
-    const int ii = p / wmax, w = p % wmax;
-    const int i = i0 + ii, I = pre + i;
-    if (w >= (I + 32) / 32) continue;
-    const int j = w * 32 + lane;
-    bool keep = false;
-    if (j <= I) {
-      keep = (i >= N - a.last_n) || (j < a.sink) || (j > I - win);
-      for (int hl = 0; hl < G; ++hl) keep |= sc[(ii * G + hl) * SPP + j] >= thr[ii * G + hl];
-    }
-    const uint32_t bits = __ballot_sync(0xFFFFFFFFu, keep);
-    if (lane == 0) {
-      a.bitmask[(static_cast<int64_t>(bo + i) * a.Hkv + g) * a.W + w] = bits;
-      atomicAdd(&cnt[ii], __popc(bits));
-    }
-  }
-  __syncthreads();
-  if (tid < nI) a.counts[static_cast<int64_t>(bo + i0 + tid) * a.Hkv + g] = cnt[tid];
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ counts, int64_t rows,
@@ -302,23 +425,20 @@ __global__ void __launch_bounds__(256) scatter_kernel(const uint32_t* __restrict
   }
 }
 
-size_t discover_smem_bytes(int D, int G, int TI, int SP) {
-  return sizeof(float) * (static_cast<size_t>(kRows) * (D + 4) + kNB * kKC * kKS +
-                          static_cast<size_t>(TI) * G * (SP + 8) + 64);
-}
+size_t discover_smem_bytes(int D) { return D == 64 ? DiscCfg<64>::SMEM_BYTES : DiscCfg<128>::SMEM_BYTES; }
 
 cudaError_t launch_discover(const DiscArgs& a, const Fp2Plan& P, int64_t items, int64_t rows, int32_t* row_ptr,
                             int32_t* col_idx, int64_t capacity, cudaStream_t stream) {
-  const size_t smem = discover_smem_bytes(a.D, a.G, a.TI, a.SP);
   cudaError_t e;
   if (a.D == 64) {
-    e = ensure_dynamic_smem(reinterpret_cast<const void*>(discover_kernel<64>), static_cast<int>(smem));
+    e = ensure_dynamic_smem(reinterpret_cast<const void*>(discover_kernel<64>), DiscCfg<64>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    discover_kernel<64><<<static_cast<unsigned>(items), kThreads, smem, stream>>>(a, P);
+    discover_kernel<64><<<static_cast<unsigned>(items), DiscCfg<64>::THREADS, DiscCfg<64>::SMEM_BYTES, stream>>>(a, P);
   } else {
-    e = ensure_dynamic_smem(reinterpret_cast<const void*>(discover_kernel<128>), static_cast<int>(smem));
+    e = ensure_dynamic_smem(reinterpret_cast<const void*>(discover_kernel<128>), DiscCfg<128>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    discover_kernel<128><<<static_cast<unsigned>(items), kThreads, smem, stream>>>(a, P);
+    discover_kernel<128><<<static_cast<unsigned>(items), DiscCfg<128>::THREADS, DiscCfg<128>::SMEM_BYTES, stream>>>(a,
+                                                                                                                 P);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   scan_kernel<<<1, 1024, 0, stream>>>(a.counts, rows, row_ptr, capacity, a.status);

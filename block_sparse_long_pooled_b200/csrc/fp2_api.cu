@@ -344,12 +344,8 @@ fp2_status run_discover(const fp2_problem* p, const fp2_sparse_params* s, const 
   a.window = s->window_blocks;
   a.last_n = s->last_n_blocks;
   a.min_sparse_len = s->min_sparse_len;
-  a.SP = std::max(32, (c.plan.max_k_nblk + 31) / 32 * 32);
-  // Largest tile of query blocks whose scores fit in shared memory (TI * G <= 32 rows).
-  int TI = std::max(1, 32 / c.G);
-  while (TI > 1 && fp2::discover_smem_bytes(a.D, c.G, TI, a.SP) > 220 * 1024) --TI;
-  if (fp2::discover_smem_bytes(a.D, c.G, TI, a.SP) > 220 * 1024)
-    return fail(FP2_ERR_UNSUPPORTED, "group size x blocks per sequence too large for discovery");
+  // One CTA computes the 128 score rows (query block, head) of TI = 128 / G query blocks.
+  const int TI = std::max(1, 128 / c.G);
   a.TI = TI;
   a.W = c.W;
   a.bitmask = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + c.off_bitmask);

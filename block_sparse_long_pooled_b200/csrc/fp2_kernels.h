@@ -35,8 +35,7 @@ struct DiscArgs {
   float ln_alpha;   // natural log of alpha (alpha > 0)
   int dense_all;    // alpha <= 0: keep everything
   int sink, window, last_n, min_sparse_len;
-  int TI;           // query blocks per CTA (TI * G <= 32)
-  int SP;           // padded score row length (>= max N, multiple of 32)
+  int TI;           // query blocks per CTA: 128 / G (the CTA's 128 score rows)
   int W;            // bitmask words per row
   uint32_t* bitmask;
   int32_t* counts;
@@ -87,7 +86,7 @@ struct AttnArgs {
 cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
 
 cudaError_t launch_pool(int dtype, const PoolArgs& a, const Fp2Plan& P, cudaStream_t stream);
-size_t discover_smem_bytes(int D, int G, int TI, int SP);
+size_t discover_smem_bytes(int D);
 cudaError_t launch_discover(const DiscArgs& a, const Fp2Plan& P, int64_t items, int64_t rows, int32_t* row_ptr,
                             int32_t* col_idx, int64_t capacity, cudaStream_t stream);
 // Returns cudaErrorInvalidValue when no kernel exists for (dtype, d, B).

@@ -189,8 +189,9 @@ def test_tiny_workload_end_to_end():
     Hn.compare_attention_full(run, inp, ora)
 
 
+# The five workloads, plus the served configuration's last-n-blocks 8 on the 64K FP8 layer.
 FULL = ["llama8b_32k_bf16", "llama8b_128k_bf16", "llama8b_128k_e4m3", "qwen30b_64k_paged_bf16",
-        "varlen6_paged_e4m3"]
+        "varlen6_paged_e4m3", "qwen4b_64k_e4m3_lastn8"]
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -228,9 +229,9 @@ def test_full_size_workloads(name):
               f"lse {r2['lse_max_abs']:.2e}")
 
 
-# More than 1024 key blocks: 32 score rows of a tile no longer fit in shared memory, so discovery
-# runs with smaller query tiles (the library picks 24, 16 and 8 rows here) and part of its warps
-# have no row; the last case is the largest sequence the ABI accepts (FP2_MAX_BLOCKS = 4096).
+# More than 1024 key blocks: discovery streams 11 to 32 key chunks of 128 blocks through each
+# CTA, twice (row maxima, then the threshold test); the last case is the largest sequence the ABI
+# accepts (FP2_MAX_BLOCKS = 4096).
 LONG = [
     small("long_g4_tile24", num_q_heads=4, num_kv_heads=1, head_dim=64, block_size=64, seqlens=(1400 * 64 - 17,),
           sink_blocks=2, window_blocks=4),
@@ -242,7 +243,7 @@ LONG = [
 
 
 @pytest.mark.parametrize("w", LONG, ids=lambda w: w.name)
-def test_long_sequences_smaller_discovery_tiles(w):
+def test_long_sequences(w):
     inp = W.generate(w)
     ora = Hn.oracle_discovery(inp, head_chunk=4)
     rp, ci = Hn.oracle_csr(ora)
