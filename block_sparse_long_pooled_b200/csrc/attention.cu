@@ -175,11 +175,11 @@ FP2_DEVICE uint32_t pruned_word(const uint32_t* kmask, int base, int i) {
 }
 
 // Bounded wait used only while draining in-flight copies at exit; ignores the abort flag.
-// Copies and MMAs complete within microseconds, so the limit is short.
-FP2_DEVICE void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status) {
+// Copies and MMAs complete within microseconds, so the limit is short (a fifth of the wait limit).
+FP2_DEVICE void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint32_t* status, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > 200000000ull) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       set_status(status, FP2_DEV_TIMEOUT);
       return;
     }
@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(384, 1)
       // they are in flight, then the remaining key tiles as ring slots free up.
       // Load p of this CTA goes to slot p % NSLOT: K of tile t is load 2t, V load 2t+1.
       auto issue_kv = [&](int jt, int j, int q, int kv) {
+        if (kv == 0 && (q >> 1) == a.withhold_k_tile) return;  // testing: this load never arrives
         const int slot = q % C::NSLOT;
         mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
         uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(384, 1)
           bool stop = false;
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = p % C::NSLOT, wrap = p / C::NSLOT;
-            if (wrap > 0 && !mbar_wait(&kv_empty[slot], (wrap - 1) & 1, abort_flag, a.status)) {
+            if (wrap > 0 && !mbar_wait(&kv_empty[slot], (wrap - 1) & 1, abort_flag, a.status, a.wait_limit_ns)) {
               stop = true;
               break;
             }
@@ -422,8 +423,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         // Never leave with copies in flight.
-        for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status);
-        for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status);
+        for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status, a.wait_limit_ns / 5);
+        for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status, a.wait_limit_ns / 5);
       }
     } else if (warp == 9 || warp == 10) {
       // ---------------------------------------------------------------- MMA issuers
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(384, 1)
       // issues each tcgen05 instruction (the *_warp wrappers).
       {
         auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-          return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, a.status));
+          return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, a.status, a.wait_limit_ns));
         };
         // Loads come in the order K(0), V(0), K(1), V(1), ...: K(j) is load 2j, V(j) load 2j+1.
         auto slot_of = [&](int q) { return q % C::NSLOT; };
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
           umma_commit_warp(mma_done);
-          if (lane == 0) mbar_wait_drain(mma_done, 0, a.status);
+          if (lane == 0) mbar_wait_drain(mma_done, 0, a.status, a.wait_limit_ns / 5);
           __syncwarp();
         } else {
           auto issue_pv = [&](int s, uint32_t vaddr, int jt) {
@@ -523,7 +524,7 @@ __global__ void __launch_bounds__(384, 1)
               umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
           }
           umma_commit_warp(pv_done);
-          if (lane == 0) mbar_wait_drain(pv_done, 0, a.status);
+          if (lane == 0) mbar_wait_drain(pv_done, 0, a.status, a.wait_limit_ns / 5);
           __syncwarp();
         }
       }
@@ -539,10 +540,10 @@ __global__ void __launch_bounds__(384, 1)
         bool ok = true;
         for (int jt = 0; jt < n_local && ok; ++jt) {
           const int qv = 2 * jt + 1, slot = qv % C::NSLOT;
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&kv_full[slot], (qv / C::NSLOT) & 1, abort_flag, a.status));
+          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&kv_full[slot], (qv / C::NSLOT) & 1, abort_flag, a.status, a.wait_limit_ns));
           if (ok && jt >= 2)
             ok = __all_sync(0xFFFFFFFFu,
-                            mbar_wait(&v16_empty[jt & 1], ((jt >> 1) - 1) & 1, abort_flag, a.status));
+                            mbar_wait(&v16_empty[jt & 1], ((jt >> 1) - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
           if (!ok) break;
           const uint8_t* src = smem + C::OFF_KV + slot * C::KV_BYTES;
           uint8_t* dst = smem + C::OFF_V16 + (jt & 1) * C::V16_BYTES;
@@ -586,12 +587,12 @@ __global__ void __launch_bounds__(384, 1)
       const float s2 = a.sm_scale_log2;
       const float bias_raw = a.log2_blk / s2;
       float m_run = -CUDART_INF_F, l_run = 0.f;
-      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status));
+      bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(mask_ready, 0, abort_flag, a.status, a.wait_limit_ns));
 
       int done_tiles = 0;
       for (int jl = 0; jl < n_local && ok; ++jl) {
         const int jt = t_begin + jl;  // position in the row's key stream
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jl & 1, abort_flag, a.status));
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jl & 1, abort_flag, a.status, a.wait_limit_ns));
         if (!ok) break;
         tc_fence_after();
         // The whole S row of this thread, in registers.
@@ -607,7 +608,7 @@ __global__ void __launch_bounds__(384, 1)
         bool pv_prev_done = jl == 0;
         auto wait_pv_prev = [&]() {
           if (!pv_prev_done) {
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (jl - 1) & 1, abort_flag, a.status));
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (jl - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
             tc_fence_after();
             pv_prev_done = true;
           }
@@ -736,7 +737,7 @@ __global__ void __launch_bounds__(384, 1)
         done_tiles = jl + 1;
       }
       if (ok && done_tiles == n_local && n_local > 0)
-        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_local - 1) & 1, abort_flag, a.status));
+        ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_local - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
       tc_fence_after();
       if (item >= 0) {
         // Piece of a split row: its normalised partial O (fp32) and natural-log LSE go to the
@@ -769,7 +770,7 @@ __global__ void __launch_bounds__(384, 1)
         const int first = item - split;  // first piece of this (row, part)
         if (qd == 0 && lane == 0) {
           int last = 0;
-          if (mbar_wait(&o_staged[s], 0, abort_flag, a.status)) {
+          if (mbar_wait(&o_staged[s], 0, abort_flag, a.status, a.wait_limit_ns)) {
             __threadfence();
             last = atomicAdd(&a.piece_cnt[first * 2 + s], 1) == nsplit - 1;
           }
@@ -777,7 +778,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(&o_merge[s]);
         }
         const bool merge =
-            __all_sync(0xFFFFFFFFu, mbar_wait(&o_merge[s], 0, abort_flag, a.status)) && merge_flag[s] != 0;
+            __all_sync(0xFFFFFFFFu, mbar_wait(&o_merge[s], 0, abort_flag, a.status, a.wait_limit_ns)) && merge_flag[s] != 0;
         if (merge && row_ok) {
           __threadfence();
           const float* lp = a.lse_slot + static_cast<int64_t>(first) * prow + s * 128 + rt;
@@ -888,7 +889,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         fence_proxy_async_smem();
         mbar_arrive(&o_staged[s]);
-        if (qd == 0 && lane == 0 && mbar_wait(&o_staged[s], 0, abort_flag, a.status) && !*abort_flag) {
+        if (qd == 0 && lane == 0 && mbar_wait(&o_staged[s], 0, abort_flag, a.status, a.wait_limit_ns) && !*abort_flag) {
           const int tok0 = P.tok_off[r] + i * BN;
           for (int hs2 = 0; hs2 < HS; ++hs2) {
             const int hl2 = (part * a.NT + s) * HS + hs2;

@@ -191,8 +191,10 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
     const int ct = tid - 128;
     const int col8 = ct % C::UPR, r0 = ct / C::UPR;
     const int chunk_off = (col8 >> 3) * (128 * 128);
-    auto convert = [&](uint8_t* hi_base, uint8_t* lo_base, auto src_of) {
-      float4 x[NU][2];
+    float4 x[NU][2];
+    // Loads of a tile's rows into registers (issued before waiting for the stage they go to, so
+    // their latency overlaps the MMAs of the chunks before), then the split and swizzled stores.
+    auto load = [&](auto src_of) {
 #pragma unroll
       for (int k = 0; k < NU; ++k) {
         const float* p = src_of(r0 + RSTEP * k);
@@ -203,6 +205,8 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
           x[k][0] = x[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+    };
+    auto store = [&](uint8_t* hi_base, uint8_t* lo_base) {
 #pragma unroll
       for (int k = 0; k < NU; ++k) {
         const int row = r0 + RSTEP * k;
@@ -216,22 +220,24 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
       __syncwarp();
     };
     const int64_t qrow0 = static_cast<int64_t>(bo + i0) * a.Hq + static_cast<int64_t>(g) * G;
-    convert(smem + C::OFF_AHI, smem + C::OFF_ALO, [&](int m) -> const float* {
+    load([&](int m) -> const float* {
       if (m >= rows) return nullptr;
       return a.qbar + (qrow0 + static_cast<int64_t>(m / G) * a.Hq + (m % G)) * D;
     });
+    store(smem + C::OFF_AHI, smem + C::OFF_ALO);
     if (lane == 0) mbar_arrive(a_full);
     for (int q = 0; q < nq; ++q) {
       const int stage = q % C::NST, use = q / C::NST;
-      if (use > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&b_empty[stage], (use - 1) & 1, abort_flag, a.status)))
-        break;
       const int j0 = (q % nch) * C::KEYS;
-      uint8_t* hb = smem + C::OFF_B + stage * 2 * C::PLANE;
-      convert(hb, hb + C::PLANE, [&](int n) -> const float* {
+      load([&](int n) -> const float* {
         const int j = j0 + n;
         if (j >= J1) return nullptr;
         return a.kbar + (static_cast<int64_t>(kbo + j) * a.Hkv + g) * D;
       });
+      if (use > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&b_empty[stage], (use - 1) & 1, abort_flag, a.status)))
+        break;
+      uint8_t* hb = smem + C::OFF_B + stage * 2 * C::PLANE;
+      store(hb, hb + C::PLANE);
       if (lane == 0) mbar_arrive(&b_full[stage]);
     }
   } else if (warp == 4 + C::NCONV) {
@@ -394,7 +400,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 __global__ void __launch_bounds__(256) scatter_kernel(const uint32_t* __restrict__ bitmask, int W,
                                                       const int32_t* __restrict__ row_ptr,
                                                       int32_t* __restrict__ col_idx, int64_t capacity, int Hkv,
-                                                      int64_t rows, const Fp2Plan P) {
+                                                      int64_t rows, const __grid_constant__ Fp2Plan P) {
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -40,6 +41,10 @@ constexpr int kMaxPieceSplits = 64;
 constexpr int64_t kAdaptiveRowCtas = 16 * 148;
 
 int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : (t == FP2_BF16 ? 2 : 1); }
+
+// Testing hooks set through fp2_debug_set (process-wide; read when attention launches).
+std::atomic<int64_t> g_wait_limit_ns{0};     // 0: the default limit of 1 s
+std::atomic<int64_t> g_withhold_k_tile{-1};  // -1: every load is issued
 
 // Everything derived from (problem, params) on the host.
 struct Ctx {
@@ -132,6 +137,21 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   P.max_k_nblk = max_k_nblk;
   for (int r = 0; r < p->num_seqs; ++r) P.sorted[r] = static_cast<int16_t>(r);
   std::stable_sort(P.sorted, P.sorted + p->num_seqs, [&](int16_t x, int16_t y) { return P.nblk[x] > P.nblk[y]; });
+  // Heavy-first work lists: per sorted position k, the items (per unit of width) of the sequences
+  // before it, for tiles of one query block and of the discovery tile.
+  P.disc_tile = std::max(1, 128 / c.G);
+  for (int t = 0; t < 2; ++t) {
+    const int tile = t == 0 ? 1 : P.disc_tile;
+    int32_t* lb = t == 0 ? P.lvl_base1 : P.lvl_base_t;
+    int64_t base = 0;
+    for (int k = 0; k < p->num_seqs; ++k) {
+      lb[k] = static_cast<int32_t>(base);
+      const int64_t hi = (P.nblk[P.sorted[k]] + tile - 1) / tile;
+      const int64_t lo = k + 1 < p->num_seqs ? (P.nblk[P.sorted[k + 1]] + tile - 1) / tile : 0;
+      base += (hi - lo) * (k + 1);
+    }
+    lb[p->num_seqs] = static_cast<int32_t>(base);
+  }
   c.T = T;
   c.Tk = Tk;
   c.total_blocks = blocks;
@@ -345,7 +365,7 @@ fp2_status run_discover(const fp2_problem* p, const fp2_sparse_params* s, const 
   a.last_n = s->last_n_blocks;
   a.min_sparse_len = s->min_sparse_len;
   // One CTA computes the 128 score rows (query block, head) of TI = 128 / G query blocks.
-  const int TI = std::max(1, 128 / c.G);
+  const int TI = c.plan.disc_tile;
   a.TI = TI;
   a.W = c.W;
   a.bitmask = reinterpret_cast<uint32_t*>(static_cast<char*>(scratch) + c.off_bitmask);
@@ -420,6 +440,9 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   a.mean_correction = s->mean_correction ? 1 : 0;
   a.total_tokens = static_cast<int>(c.T);
   a.status = status_ptr(scratch);
+  const int64_t lim = g_wait_limit_ns.load();
+  a.wait_limit_ns = lim > 0 ? static_cast<uint64_t>(lim) : 1000000000ull;
+  a.withhold_k_tile = static_cast<int>(g_withhold_k_tile.load());
   {
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -596,6 +619,22 @@ fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_out) {
   if (w & (FP2_DEV_PAGE_OOB | FP2_DEV_INDEX_OOB | FP2_DEV_CAPACITY))
     return fail(FP2_ERR_DEVICE_BOUNDS, "device reported an out-of-range page id, index entry or capacity overflow");
   return FP2_OK;
+}
+
+fp2_status fp2_debug_set(int32_t key, int64_t value) {
+  switch (key) {
+    case FP2_DEBUG_WAIT_LIMIT_NS:
+      if (value != 0 && (value < 100000 || value > 10000000000LL))
+        return fail(FP2_ERR_INVALID_ARG, "wait limit must be 0 (default) or in [1e5, 1e10] ns");
+      g_wait_limit_ns.store(value);
+      return FP2_OK;
+    case FP2_DEBUG_WITHHOLD_K_TILE:
+      if (value < -1 || value > FP2_MAX_BLOCKS) return fail(FP2_ERR_INVALID_ARG, "tile must be -1 or in [0, FP2_MAX_BLOCKS]");
+      g_withhold_k_tile.store(value);
+      return FP2_OK;
+    default:
+      return fail(FP2_ERR_INVALID_ARG, "unknown debug key");
+  }
 }
 
 const char* fp2_last_error(void) { return g_last_error.c_str(); }

@@ -27,39 +27,47 @@ FP2_DEVICE void set_status(uint32_t* status, uint32_t bits) { atomicOr(status, b
 
 // Work item v of a list ordered by level descending (level = query block or query-block tile),
 // `width` items per (sequence, level), sequences with fewer levels dropping out as the level
-// falls.  nlev(r) = ceil(nblk[r] / tile).  Returns false when v is past the end.
+// falls.  nlev(r) = ceil(nblk[r] / tile); tile is 1 or P.disc_tile (the two tables the host
+// builds).  The segment of the k-th sequence in `sorted` order is found by binary search over
+// its precomputed start.  Returns false when v is past the end.
 FP2_DEVICE bool map_heavy_first(const Fp2Plan& P, int tile, int width, long long v, int& r, int& lvl, int& sub) {
-  long long base = 0;
-  for (int k = 0; k < P.num_seqs; ++k) {
-    const int hi = (P.nblk[P.sorted[k]] + tile - 1) / tile;
-    const int lo = (k + 1 < P.num_seqs) ? (P.nblk[P.sorted[k + 1]] + tile - 1) / tile : 0;
-    const long long per_level = static_cast<long long>(k + 1) * width;
-    const long long cnt = static_cast<long long>(hi - lo) * per_level;
-    if (v < base + cnt) {
-      const long long off = v - base;
-      lvl = hi - 1 - static_cast<int>(off / per_level);
-      const int rem = static_cast<int>(off % per_level);
-      r = P.sorted[rem / width];
-      sub = rem % width;
-      return true;
-    }
-    base += cnt;
+  const int32_t* lb = tile == 1 ? P.lvl_base1 : P.lvl_base_t;
+  const int n = P.num_seqs;
+  if (v < 0 || v >= static_cast<long long>(lb[n]) * width) return false;
+  int lo_k = 0, hi_k = n - 1;  // the last k with lb[k] * width <= v
+  while (lo_k < hi_k) {
+    const int mid = (lo_k + hi_k + 1) >> 1;
+    if (static_cast<long long>(lb[mid]) * width <= v) lo_k = mid; else hi_k = mid - 1;
   }
-  return false;
+  const int k = lo_k;
+  const int hi = (P.nblk[P.sorted[k]] + tile - 1) / tile;
+  const long long per_level = static_cast<long long>(k + 1) * width;
+  const long long off = v - static_cast<long long>(lb[k]) * width;
+  lvl = hi - 1 - static_cast<int>(off / per_level);
+  const int rem = static_cast<int>(off % per_level);
+  r = P.sorted[rem / width];
+  sub = rem % width;
+  return true;
 }
 
-// Sequence of query block b.
+// Sequence of query block b (the last sequence whose first block is <= b).
 FP2_DEVICE int seq_of_block(const Fp2Plan& P, int b) {
-  int r = 0;
-  while (r + 1 < P.num_seqs && P.blk_off[r + 1] <= b) ++r;
-  return r;
+  int lo = 0, hi = P.num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.blk_off[mid] <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 // Sequence of key block b.
 FP2_DEVICE int seq_of_key_block(const Fp2Plan& P, int b) {
-  int r = 0;
-  while (r + 1 < P.num_seqs && P.k_blk_off[r + 1] <= b) ++r;
-  return r;
+  int lo = 0, hi = P.num_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.k_blk_off[mid] <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 // ------------------------------------------------------------------ mbarrier
@@ -98,9 +106,9 @@ FP2_DEVICE void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// Bounded wait: gives up after kWaitLimitNs of wall time (or at once when another role of the
-// CTA already gave up), records FP2_DEV_TIMEOUT and returns false.  Nothing in this library
-// waits without a limit.
+// Bounded wait: gives up after limit_ns of wall time (kWaitLimitNs unless the launch passes its
+// own), or at once when another role of the CTA already gave up; records FP2_DEV_TIMEOUT and
+// returns false.  Nothing in this library waits without a limit.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 // Non-blocking probe of the phase (no suspend): the cheap first check of a wait that is often
@@ -117,14 +125,15 @@ FP2_DEVICE bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-FP2_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
+FP2_DEVICE bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* status,
+                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_test_wait(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       set_status(status, FP2_DEV_TIMEOUT);
       return false;

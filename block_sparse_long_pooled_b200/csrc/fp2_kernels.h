@@ -78,6 +78,8 @@ struct AttnArgs {
   float* o_slot;              // [adapt, NT * 128, d] f32 normalised partial outputs of the pieces
   float* lse_slot;            // [adapt, NT * 128] f32 natural-log partial LSE
   uint32_t* status;
+  uint64_t wait_limit_ns;     // limit of every mbarrier wait (drains of in-flight copies: a fifth)
+  int withhold_k_tile;        // testing: the producer skips the K load of this local key tile (-1: none)
 };
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device.  The

@@ -67,7 +67,8 @@ FP2_DEVICE void accumulate(const uint4& v, float* acc) {
 // kbar/vbar row b (skipped for prefix blocks when they are already pooled); when J lies in the
 // query chunk its Q rows are pooled into qbar row blk_off[r] + (J - pre_blk[r]).
 template <int DT>
-__global__ void __launch_bounds__(256) pool_kernel(const PoolArgs a, const Fp2Plan P) {
+__global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolArgs a,
+                                                   const __grid_constant__ Fp2Plan P) {
   constexpr int VEC = 16 / Elt<DT>::kBytes;  // elements per 16-byte vector
   const int b = blockIdx.x;
   const int r = seq_of_key_block(P, b);

@@ -21,13 +21,14 @@ FP2_OK, FP2_ERR_INVALID_ARG, FP2_ERR_UNSUPPORTED, FP2_ERR_WORKSPACE_TOO_SMALL = 
 FP2_ERR_CUDA, FP2_ERR_DEVICE_BOUNDS, FP2_ERR_TIMEOUT = 4, 5, 6
 FP2_F32, FP2_BF16, FP2_E4M3 = 0, 1, 2
 FP2_DEV_PAGE_OOB, FP2_DEV_INDEX_OOB, FP2_DEV_CAPACITY, FP2_DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
-FP2_MAX_SEQS, FP2_MAX_BLOCKS = 128, 4096
+FP2_MAX_SEQS, FP2_MAX_BLOCKS = 512, 4096
 
 STATUS_NAMES = {0: "FP2_OK", 1: "FP2_ERR_INVALID_ARG", 2: "FP2_ERR_UNSUPPORTED", 3: "FP2_ERR_WORKSPACE_TOO_SMALL",
                 4: "FP2_ERR_CUDA", 5: "FP2_ERR_DEVICE_BOUNDS", 6: "FP2_ERR_TIMEOUT"}
 
 EXPORTED = ("fp2_workspace_query", "fp2_workspace_size", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
-            "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static")
+            "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static", "fp2_debug_set")
+FP2_DEBUG_WAIT_LIMIT_NS, FP2_DEBUG_WITHHOLD_K_TILE = 1, 2
 FP2_STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -107,6 +108,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fp2_workspace_query", "fp2_workspace_size", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
                  "fp2_get_device_status", "fp2_discover_static"):
         getattr(lib, name).restype = ctypes.c_int
+    lib.fp2_debug_set.argtypes = [ctypes.c_int32, ctypes.c_int64]
+    lib.fp2_debug_set.restype = ctypes.c_int
     lib.fp2_last_error.argtypes = []
     lib.fp2_last_error.restype = ctypes.c_char_p
     lib.fp2_version.argtypes = []
@@ -246,6 +249,11 @@ def fp2_get_device_status(scratch) -> tuple:
     bits = ctypes.c_uint32(0)
     st = load_library().fp2_get_device_status(_ptr(scratch), ctypes.byref(bits))
     return st, int(bits.value)
+
+
+def fp2_debug_set(key: int, value: int):
+    """Testing hook (process-wide): FP2_DEBUG_WAIT_LIMIT_NS or FP2_DEBUG_WITHHOLD_K_TILE."""
+    _check(load_library().fp2_debug_set(int(key), int(value)))
 
 
 def fp2_last_error() -> str:

@@ -70,7 +70,7 @@ extern "C" {
 #define FP2_API
 #endif
 
-#define FP2_MAX_SEQS 128
+#define FP2_MAX_SEQS 512
 #define FP2_MAX_BLOCKS 4096
 
 typedef enum {
@@ -237,6 +237,21 @@ FP2_API fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_o
 FP2_API fp2_status fp2_discover_static(const fp2_problem* problem, const fp2_sparse_params* params,
                                        const fp2_pooled* pooled, const fp2_index* index, uint32_t* status_dev,
                                        fp2_stream_t stream);
+
+/* Testing hooks, process-wide, for exercising the device-side time limits without a GPU fault.
+ * Not for production use.  The paper has no counterpart.
+ *   FP2_DEBUG_WAIT_LIMIT_NS    limit of every wait inside the attention kernel, in ns (0 restores
+ *                              the default of 1 s; otherwise 1e5 .. 1e10); draining copies in
+ *                              flight at exit waits up to a fifth of it.
+ *   FP2_DEBUG_WITHHOLD_K_TILE  the producer of every attention CTA skips the K load of its local
+ *                              key tile `value` (-1 restores normal operation): that tile's barrier
+ *                              never completes, the wait for it runs out, every role of the CTA
+ *                              gives up and drains through its bounded paths, and the status word
+ *                              gets FP2_DEV_TIMEOUT.  Nothing faults; the next call is unaffected.
+ * Returns FP2_ERR_INVALID_ARG for an unknown key or a value out of range. */
+#define FP2_DEBUG_WAIT_LIMIT_NS 1
+#define FP2_DEBUG_WITHHOLD_K_TILE 2
+FP2_API fp2_status fp2_debug_set(int32_t key, int64_t value);
 
 /* Message for the last failing call on this thread ("" if none). */
 FP2_API const char* fp2_last_error(void);

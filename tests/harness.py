@@ -276,9 +276,13 @@ def seq_group_kv(inp: W.Inputs, r: int, g: int):
     if inp.page_table is None:
         return inp.dequant("k", heads=[g], tokens=slice(a, b)), inp.dequant("v", heads=[g], tokens=slice(a, b))
     L = b - a
-    pt = inp.page_table[r:r + 1]
-    kc = inp.k_cache[:, :, g:g + 1].to(torch.float64).numpy() * inp.k_descale
-    vc = inp.v_cache[:, :, g:g + 1].to(torch.float64).numpy() * inp.v_descale
+    ps = inp.k_cache.shape[1]
+    pages = inp.page_table[r, :-(-L // ps)]
+    # the sequence's own pages, renumbered 0..n-1, then the oracle's page-table gather
+    idx = torch.from_numpy(pages.astype(np.int64))
+    kc = inp.k_cache[idx][:, :, g:g + 1].to(torch.float64).numpy() * inp.k_descale
+    vc = inp.v_cache[idx][:, :, g:g + 1].to(torch.float64).numpy() * inp.v_descale
+    pt = np.arange(len(pages), dtype=np.int32)[None, :]
     return O.gather_paged(kc, pt, [L]), O.gather_paged(vc, pt, [L])
 
 

@@ -178,3 +178,26 @@ def _load_fresh(path):
         return fp2.load_library(path)
     finally:
         fp2._lib = saved
+
+
+def test_debug_hooks_validate_and_reset():
+    with pytest.raises(fp2.FP2Error):
+        fp2.fp2_debug_set(99, 0)
+    with pytest.raises(fp2.FP2Error):
+        fp2.fp2_debug_set(fp2.FP2_DEBUG_WAIT_LIMIT_NS, 10)           # below 0.1 ms
+    with pytest.raises(fp2.FP2Error):
+        fp2.fp2_debug_set(fp2.FP2_DEBUG_WITHHOLD_K_TILE, -2)
+    fp2.fp2_debug_set(fp2.FP2_DEBUG_WAIT_LIMIT_NS, 2_000_000)
+    fp2.fp2_debug_set(fp2.FP2_DEBUG_WAIT_LIMIT_NS, 0)
+    fp2.fp2_debug_set(fp2.FP2_DEBUG_WITHHOLD_K_TILE, 3)
+    fp2.fp2_debug_set(fp2.FP2_DEBUG_WITHHOLD_K_TILE, -1)
+
+
+def test_sequence_count_limit():
+    ok = _problem(seqlens=(3,) * fp2.FP2_MAX_SEQS, Hq=4, Hkv=2)
+    ws = fp2.fp2_workspace_query(ok, fp2.make_params(64))
+    assert ws.index_rows == fp2.FP2_MAX_SEQS * 2
+    too_many = _problem(seqlens=(3,) * (fp2.FP2_MAX_SEQS + 1), Hq=4, Hkv=2)
+    with pytest.raises(fp2.FP2Error) as e:
+        fp2.fp2_workspace_query(too_many, fp2.make_params(64))
+    assert e.value.status == fp2.FP2_ERR_UNSUPPORTED

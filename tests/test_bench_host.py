@@ -1,5 +1,5 @@
-"""Host-side helpers of bench.py that feed its JSON line (no GPU): the fp32 FMA peak used for the
-discovery roofline and the kernel-launch count per step."""
+"""Host-side helpers of bench.py that feed its JSON line (no GPU): the peaks of the discovery and
+Stage-1 rooflines and the kernel-launch count per step."""
 
 import numpy as np
 import torch
@@ -9,10 +9,19 @@ from block_sparse_long_pooled_b200 import fp2
 from synth import workloads as W
 
 
-def test_fp32_fma_peak_from_unit_counts():
-    # 148 SMs x 128 FMA lanes x 2 flops x clock
-    assert abs(bench.fp32_fma_peak_tflops({"sm_max_mhz": 1965.0}) - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
-    assert bench.fp32_fma_peak_tflops(None) == bench.fp32_fma_peak_tflops({"sm_max_mhz": 1965.0})
+def test_stage1_rooflines_from_peaks_and_stage_times():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1400.0, "source": "test"}
+    assert bench.discover_peak_tflops(peaks) == 500.0      # three bf16 products per fp32-accurate one
+
+    class P:
+        def discover_flops(self):
+            return 5e12 * 1e-4                              # 5 TFLOP/s over 0.1 ms
+
+        def pool_bytes(self):
+            return 6000e9 * 0.3e-3 * 0.5                    # half of HBM over 0.3 ms
+    d, st1 = bench.rooflines_stage1(P(), {"pool": 0.2, "discover": 0.1, "attend": 1.0}, peaks)
+    assert abs(d["achieved"] - 5.0) < 1e-9 and abs(d["frac"] - 0.01) < 1e-12 and d["bound"] == "tensor"
+    assert abs(st1["frac"] - 0.5) < 1e-12 and st1["bound"] == "hbm"
 
 
 class _FakePath:

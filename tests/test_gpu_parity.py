@@ -162,6 +162,27 @@ def test_adaptive_splits_automatic_on_a_mixed_batch():
     Hn.compare_attention_pairs(run, inp, Hn.oracle_pairs(inp, ora, pairs))
 
 
+def test_continuous_batch_of_301_requests():
+    """A continuous batch above the former 128-request limit: 300 short requests of 1 to 600 tokens
+    and one 20K-token request, paged; the whole index and whole pairs of every request's first and
+    last blocks (and the long request's needle and heaviest rows) against the oracle."""
+    rng = np.random.default_rng(5)
+    lens = tuple(int(x) for x in rng.integers(1, 601, size=300)) + (20000,)
+    w = small("batch301_paged", seqlens=lens, num_q_heads=8, num_kv_heads=2, paged=True, page_size=64,
+              sink_blocks=2, window_blocks=4, min_sparse_len=256)
+    inp = W.generate(w)
+    ora = Hn.oracle_discovery(inp)
+    rp, ci = Hn.oracle_csr(ora)
+    run = Hn.run_gpu(inp, external_index=(rp, ci))
+    Hn.compare_pooled(run, inp, ora)
+    stats = Hn.compare_index(run, inp, ora)
+    pairs = Hn.select_pairs(inp, ora, n_random=0)
+    Hn.compare_attention_pairs(run, inp, Hn.oracle_pairs(inp, ora, pairs))
+    if stats["borderline_mismatches"] == 0:
+        run2 = Hn.run_gpu(inp)
+        Hn.compare_attention_pairs(run2, inp, Hn.oracle_pairs(inp, ora, pairs))
+
+
 def test_tiny_workload_end_to_end():
     """The 1K fp32 workload with its four planted needle blocks, through fp2_prefill."""
     import torch
