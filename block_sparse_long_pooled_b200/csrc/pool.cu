@@ -3,11 +3,11 @@
 // simple average of its tokens).
 //
 // One pass over Q, K and V.  A CTA owns one pooled block b (B consecutive tokens of one
-// sequence) and a 256-vector slice of the concatenated token row [Q row | K row | V row];
+// sequence) and a 128-vector slice of the concatenated token row [Q row | K row | V row];
 // each thread owns one 16-byte column vector of that row and walks the block's tokens
 // with eight independent 16-byte streaming loads in flight, accumulating in fp32.  Paged
-// K/V rows are gathered through the page table.  HBM-bound: the only traffic is one read
-// of Q, K, V and a (1/B)-sized write of the means.
+// K/V rows are gathered through the page table, whose entries for the block are read once per
+// CTA.  HBM-bound: the only traffic is one read of Q, K, V and a (1/B)-sized write of the means.
 #include "fp2_device.cuh"
 #include "fp2_kernels.h"
 
@@ -63,11 +63,12 @@ FP2_DEVICE void accumulate(const uint4& v, float* acc) {
   }
 }
 
-// One CTA per key block b (absolute block J of sequence r).  Its K and V rows are pooled into
+// One CTA per (key block b, slice of 128 vectors of the token row); block b is absolute block J
+// of sequence r.  Its K and V rows are pooled into
 // kbar/vbar row b (skipped for prefix blocks when they are already pooled); when J lies in the
 // query chunk its Q rows are pooled into qbar row blk_off[r] + (J - pre_blk[r]).
 template <int DT>
-__global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolArgs a,
+__global__ void __launch_bounds__(128) pool_kernel(const __grid_constant__ PoolArgs a,
                                                    const __grid_constant__ Fp2Plan P) {
   constexpr int VEC = 16 / Elt<DT>::kBytes;  // elements per 16-byte vector
   const int b = blockIdx.x;
@@ -79,6 +80,26 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolA
   const int n = min(a.B, Lk - t0);
   const int VQ = a.Hq * a.D / VEC, VK = a.Hkv * a.D / VEC;
   const int vid = blockIdx.y * blockDim.x + threadIdx.x;
+  // Paged K/V: the block's page ids (B / page_size of them, at most 8 since page_size >= 16, or
+  // one page holding the whole block) are read from the page table once per CTA, so the token
+  // loop below issues no dependent page-table loads.  Every thread reaches the barrier.
+  __shared__ int pg_s[8];
+  if (a.page_table != nullptr) {
+    const int np = a.page_size >= a.B ? 1 : a.B / a.page_size;
+    if (threadIdx.x < np) {
+      const int tl = t0 + static_cast<int>(threadIdx.x) * a.page_size;
+      int page = 0;
+      if (tl < Lk) {
+        page = a.page_table[static_cast<int64_t>(r) * a.max_pages + tl / a.page_size];
+        if (page < 0 || page >= a.num_pages) {
+          set_status(a.status, FP2_DEV_PAGE_OOB);
+          page = 0;
+        }
+      }
+      pg_s[threadIdx.x] = page;
+    }
+    __syncthreads();
+  }
   if (vid >= VQ + 2 * VK || n <= 0) return;
 
   int which, col;
@@ -106,26 +127,16 @@ __global__ void __launch_bounds__(256) pool_kernel(const __grid_constant__ PoolA
   for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
 
   for (int t = 0; t < n; t += 8) {
+    // Tokens t .. t+7 share one page (page_size >= 16 is a multiple of 8).
+    int64_t row0 = tok_base + t;
+    if (paged) {
+      const int pslot = a.page_size >= a.B ? 0 : t / a.page_size;
+      row0 = static_cast<int64_t>(pg_s[pslot]) * a.page_size + ((t0 + t) % a.page_size);
+    }
     uint4 buf[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int tt = t + u;
-      if (tt < n) {
-        int64_t rowidx;
-        if (paged) {
-          const int tl = t0 + tt;
-          int page = a.page_table[static_cast<int64_t>(r) * a.max_pages + tl / a.page_size];
-          if (page < 0 || page >= a.num_pages) {
-            set_status(a.status, FP2_DEV_PAGE_OOB);
-            page = 0;
-          }
-          rowidx = static_cast<int64_t>(page) * a.page_size + (tl % a.page_size);
-        } else {
-          rowidx = tok_base + tt;
-        }
-        buf[u] = ld_stream_v4(base + (rowidx * stride + col) * Elt<DT>::kBytes);
-      }
-    }
+    for (int u = 0; u < 8; ++u)
+      if (t + u < n) buf[u] = ld_stream_v4(base + ((row0 + u) * stride + col) * Elt<DT>::kBytes);
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       if (t + u < n) accumulate<DT>(buf[u], acc);
@@ -169,13 +180,15 @@ cudaError_t launch_pool(int dtype, const PoolArgs& a, const Fp2Plan& P, cudaStre
   const int elt = dtype == FP2_F32 ? 4 : (dtype == FP2_BF16 ? 2 : 1);
   const int vec = 16 / elt;
   const int nvec = (a.Hq + 2 * a.Hkv) * a.D / vec;
-  dim3 grid(P.total_k_blocks, (nvec + 255) / 256);
+  // 128 threads per CTA: the vector counts of the usual head layouts ((Hq + 2 Hkv) x d / vector)
+  // are multiples of 128, so no CTA carries idle threads.
+  dim3 grid(P.total_k_blocks, (nvec + 127) / 128);
   if (dtype == FP2_F32)
-    pool_kernel<0><<<grid, 256, 0, stream>>>(a, P);
+    pool_kernel<0><<<grid, 128, 0, stream>>>(a, P);
   else if (dtype == FP2_BF16)
-    pool_kernel<1><<<grid, 256, 0, stream>>>(a, P);
+    pool_kernel<1><<<grid, 128, 0, stream>>>(a, P);
   else
-    pool_kernel<2><<<grid, 256, 0, stream>>>(a, P);
+    pool_kernel<2><<<grid, 128, 0, stream>>>(a, P);
   return cudaGetLastError();
 }
 
