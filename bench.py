@@ -616,7 +616,7 @@ def chunked_sweep(args, dev, peaks):
     full = fp2.make_problem(q, k, v, [0, L], w.num_kv_heads)
     ws_full = fp2.fp2_workspace_query(full, params)
     _, pooled = fp2.alloc_pooled(ws_full, full, dev)
-    pst = fp2.fp2_pooled(*(pooled[n].data_ptr() for n in ("qbar", "kbar", "vbar", "kbar_mma", "vbar_mma")))
+    pst = fp2.pooled_struct(pooled)
     scratch = fp2.alloc_scratch(ws_full.prefill_scratch_bytes, dev)
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
     lines = []

@@ -38,8 +38,11 @@
 //                    and the tensor pipe interleaves them; one issuer would stall the pipe at
 //                    every wait between groups.  Both issue tcgen05.mma from lane 0 and signal
 //                    mbarriers with tcgen05.commit.
-//   warp 11          e4m3 inputs: converts each V tile to f16 in shared memory for the f16 PV
-//                    product; otherwise idle (it completes warpgroup 2 for the register split).
+//   warp 11          idle (it completes warpgroup 2 for the register split).
+// e4m3 inputs: QK runs on the e4m3 Q and K tiles; V tiles come from the exact f16 copy of V that
+// the pooling pass writes (and the mean-correction vbar tiles from its f16 means), so PV is an f16
+// product with P written as f16.  Converting V here instead would redo it for every row that keeps
+// a block (about 74 times per tile at 128K) on one warp's conversion pipe.
 // TMEM: S | P0 | P1 | O0 | O1.  One S buffer serves both M tiles in turn: a softmax warpgroup
 // copies its S tile into registers and releases the buffer before doing any arithmetic, so
 // the next QK product (the other tile's, or this tile's next key tile) is computed while the
@@ -67,13 +70,16 @@ struct AttnCfg {
   static constexpr int UK = 32 / ELT;    // K extent of one MMA instruction (32 bytes)
   static constexpr int BM = 128;
   static constexpr int Q_BYTES = BM * D * ELT;
-  static constexpr int KV_BYTES = BN * D * ELT;
-  // e4m3: QK runs on e4m3 operands; V tiles are converted to f16 in shared memory (exact) and PV
-  // runs as an f16 MMA with P written as f16.  V16 holds two converted tiles.
+  // e4m3: QK runs on e4m3 operands; the V side (V tiles and vbar tiles) is f16, PV an f16 MMA.
   static constexpr bool V16 = DT == 2;
-  static constexpr int V16_BYTES = V16 ? BN * D * 2 : 0;
+  static constexpr int VELT = V16 ? 2 : ELT;        // bytes per V element
+  static constexpr int VKCH = 128 / VELT;           // V elements in one 128-byte swizzled row
+  static constexpr int VDCH = D / VKCH;             // 128-byte chunks of a V row
+  static constexpr int K_BYTES = BN * D * ELT;      // one K (or kbar) tile
+  static constexpr int V_BYTES = BN * D * VELT;     // one V (or vbar) tile
+  static constexpr int KV_BYTES = K_BYTES > V_BYTES ? K_BYTES : V_BYTES;  // ring slot
   static constexpr int TILE_BUDGET = 200 * 1024;
-  static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES - 2 * V16_BYTES) / KV_BYTES;
+  static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES) / KV_BYTES;
   static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
   // PV operand type: f16 for e4m3 inputs, else the input type; K extent of one PV MMA.
   static constexpr int PV_KIND = V16 ? 1 : KIND;
@@ -99,9 +105,8 @@ struct AttnCfg {
   static constexpr uint32_t IDESC_PV = make_idesc(PV_FMT, PV_FMT, 0, 1, 128, D);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
-  static constexpr int OFF_V16 = OFF_KV + NSLOT * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V16 + 2 * V16_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 4 + 2;
+  static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 2;
   // Output staging for TMA stores: tile s's normalised O (128 rows x d, output type) goes into
   // the shared memory of its own Q tile, free once the tile's last QK product is done; only when
   // it fits there (bf16 and f32 inputs; e4m3 Q tiles are half the size of a bf16 O tile).
@@ -205,9 +210,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* s_free = mma_done + 1;  // [2]: the S buffer has been copied out by softmax s
   uint64_t* pv_done = s_free + 2;   // the PV issuer's final commit
   uint64_t* o_staged = pv_done + 1; // [2]: every row of tile s is staged for the TMA store
-  uint64_t* v16_full = o_staged + 2;   // [2]: converted f16 V tile ready (e4m3 inputs)
-  uint64_t* v16_empty = v16_full + 2;  // [2]: its PV products are done
-  uint64_t* o_merge = v16_empty + 2;   // [2]: piece CTAs: the tile's merge decision is in merge_flag
+  uint64_t* o_merge = o_staged + 2;    // [2]: piece CTAs: the tile's merge decision is in merge_flag
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
@@ -267,8 +270,6 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&o_done[s], 1);
       mbar_init(&s_free[s], 128);
       mbar_init(&o_staged[s], 128);
-      mbar_init(&v16_full[s], 1);
-      mbar_init(&v16_empty[s], 1);
       mbar_init(&o_merge[s], 1);
     }
     for (int k = 0; k < C::NSLOT; ++k) {
@@ -299,16 +300,18 @@ __global__ void __launch_bounds__(384, 1)
       auto issue_kv = [&](int jt, int j, int q, int kv) {
         if (kv == 0 && (q >> 1) == a.withhold_k_tile) return;  // testing: this load never arrives
         const int slot = q % C::NSLOT;
-        mbar_arrive_expect_tx(&kv_full[slot], C::KV_BYTES);
+        // K side in the input type; V side in the PV operand type (f16 for e4m3 inputs).
+        const int dch = kv ? C::VDCH : C::DCH, kch = kv ? C::VKCH : C::KCH;
+        mbar_arrive_expect_tx(&kv_full[slot], kv ? C::V_BYTES : C::K_BYTES);
         uint8_t* dst = smem + C::OFF_KV + slot * C::KV_BYTES;
         if (j < 0) {
           const CUtensorMap* tm = kv ? &a.tm_vb : &a.tm_kb;
-          for (int c = 0; c < C::DCH; ++c)
-            tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_blk_off[r] + jt * BN);
-        } else if (a.page_table == nullptr) {
+          for (int c = 0; c < dch; ++c)
+            tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * kch, g, P.k_blk_off[r] + jt * BN);
+        } else if (a.page_table == nullptr || (kv && a.v_contig)) {
           const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
-          for (int c = 0; c < C::DCH; ++c)
-            tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * C::KCH, g, P.k_tok_off[r] + j * BN);
+          for (int c = 0; c < dch; ++c)
+            tma_load_3d(dst + c * (BN * 128), tm, &kv_full[slot], c * kch, g, P.k_tok_off[r] + j * BN);
         } else {
           const CUtensorMap* tm = kv ? &a.tm_v : &a.tm_k;
           const int PR = min(BN, a.page_size);
@@ -507,68 +510,19 @@ __global__ void __launch_bounds__(384, 1)
           };
           for (int jt = 0; jt < n_local && ok; ++jt) {
             const int qv = 2 * jt + 1;
-            uint32_t vaddr;
-            if constexpr (C::V16) {
-              if (!(ok = wait_all(&v16_full[jt & 1], (jt >> 1) & 1))) break;
-              vaddr = sbase + C::OFF_V16 + (jt & 1) * C::V16_BYTES;
-            } else {
-              if (!(ok = kv_wait(qv))) break;
-              vaddr = slot_addr(qv);
-            }
+            if (!(ok = kv_wait(qv))) break;
+            const uint32_t vaddr = slot_addr(qv);
             for (int s = 0; s < a.NT; ++s) {
               if (!(ok = wait_all(&p_full[s], jt & 1))) break;
               tc_fence_after();
               issue_pv(s, vaddr, jt);
             }
             if (!ok) break;
-            if constexpr (C::V16)
-              umma_commit_warp(&v16_empty[jt & 1]);  // converted V(jt) fully consumed
-            else
-              umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
+            umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
           }
           umma_commit_warp(pv_done);
           if (lane == 0) mbar_wait_drain(pv_done, 0, a.status, a.wait_limit_ns / 5);
           __syncwarp();
-        }
-      }
-    } else if (warp == 11) {
-      if constexpr (C::V16) {
-        // ---------------------------------------------------------------- V converter (e4m3)
-        // Each V tile (BN keys x 128 e4m3, 128-byte swizzled rows) becomes an f16 tile in the
-        // layout the PV MMA reads (two 64-column chunks of BN rows x 128 bytes, swizzled); exact,
-        // since every e4m3 value is an f16 value.  The ring slot is released once it is read.
-        // Source row j: 16-byte unit u holds d 16u .. 16u+15 at position u ^ (j & 7).
-        // Destination chunk c, row j: 16-byte unit u holds d 64c + 8u .. +7 at position u ^ (j & 7).
-        static_assert(D == 128, "the e4m3 V converter assumes d = 128");
-        bool ok = true;
-        for (int jt = 0; jt < n_local && ok; ++jt) {
-          const int qv = 2 * jt + 1, slot = qv % C::NSLOT;
-          ok = __all_sync(0xFFFFFFFFu, mbar_wait(&kv_full[slot], (qv / C::NSLOT) & 1, abort_flag, a.status, a.wait_limit_ns));
-          if (ok && jt >= 2)
-            ok = __all_sync(0xFFFFFFFFu,
-                            mbar_wait(&v16_empty[jt & 1], ((jt >> 1) - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
-          if (!ok) break;
-          const uint8_t* src = smem + C::OFF_KV + slot * C::KV_BYTES;
-          uint8_t* dst = smem + C::OFF_V16 + (jt & 1) * C::V16_BYTES;
-  #pragma unroll 2
-          for (int x = lane; x < BN * 8; x += 32) {
-            const int j = x >> 3, u = x & 7;
-            const uint4 w = *reinterpret_cast<const uint4*>(src + j * 128 + ((u ^ (j & 7)) << 4));
-            const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x & 0xFFFFu), e4m3x2_to_f16x2(w.x >> 16),
-                                        e4m3x2_to_f16x2(w.y & 0xFFFFu), e4m3x2_to_f16x2(w.y >> 16));
-            const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z & 0xFFFFu), e4m3x2_to_f16x2(w.z >> 16),
-                                        e4m3x2_to_f16x2(w.w & 0xFFFFu), e4m3x2_to_f16x2(w.w >> 16));
-            const int c = u >> 2, u0 = 2 * (u & 3);
-            uint8_t* rowp = dst + c * (BN * 128) + j * 128;
-            *reinterpret_cast<uint4*>(rowp + ((u0 ^ (j & 7)) << 4)) = lo;
-            *reinterpret_cast<uint4*>(rowp + (((u0 + 1) ^ (j & 7)) << 4)) = hi;
-          }
-          fence_proxy_async_smem();  // the tensor core reads the tile through the async proxy
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&kv_empty[slot]);
-            mbar_arrive(&v16_full[jt & 1]);
-          }
         }
       }
     }

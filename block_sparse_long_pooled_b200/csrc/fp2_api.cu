@@ -40,7 +40,10 @@ constexpr int kMaxPieceSplits = 64;
 // and there the plan kernel and the idle piece CTAs would cost a few percent.
 constexpr int64_t kAdaptiveRowCtas = 16 * 148;
 
-int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : (t == FP2_BF16 ? 2 : 1); }
+// f16 operands exist only inside the library (the V side of E4M3 attention); it is no input dtype.
+constexpr fp2_dtype kOperandF16 = static_cast<fp2_dtype>(100);
+
+int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : ((t == FP2_BF16 || t == kOperandF16) ? 2 : 1); }
 
 // Testing hooks set through fp2_debug_set (process-wide; read when attention launches).
 std::atomic<int64_t> g_wait_limit_ns{0};     // 0: the default limit of 1 s
@@ -60,7 +63,8 @@ struct Ctx {
   int pieces = 0, piece_tiles = 0;          // piece capacity; forced piece size (0 = automatic)
   size_t off_item0 = 0, off_items = 0, off_nitems = 0, off_pcnt = 0, off_oslot = 0, off_lslot = 0;
   // fp2_prefill carve-outs (offsets after scratch_bytes)
-  size_t off_qbar = 0, off_kbar = 0, off_vbar = 0, off_kbm = 0, off_vbm = 0, off_rowptr = 0, off_colidx = 0;
+  size_t off_qbar = 0, off_kbar = 0, off_vbar = 0, off_kbm = 0, off_vbm = 0, off_v16 = 0, off_rowptr = 0,
+         off_colidx = 0;
 };
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -192,7 +196,10 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   w.kbar_bytes = static_cast<size_t>(kblocks) * Hkv * D * 4;
   w.vbar_bytes = w.kbar_bytes;
   w.kbar_mma_bytes = static_cast<size_t>(kblocks) * Hkv * D * c.elt;
-  w.vbar_mma_bytes = w.kbar_mma_bytes;
+  // The V-side operands of the PV product are f16 for E4M3 inputs (pooled vbar and the V copy).
+  const bool e4 = p->dtype == FP2_E4M3;
+  w.vbar_mma_bytes = static_cast<size_t>(kblocks) * Hkv * D * (e4 ? 2 : c.elt);
+  w.v16_bytes = e4 ? static_cast<size_t>(Tk) * Hkv * D * 2 : 0;
   w.row_ptr_bytes = static_cast<size_t>(c.rows + 1) * 4;
   w.col_idx_bytes = static_cast<size_t>(std::max<int64_t>(cap, 1)) * 4;
   // Attention launch shape: M tiles of 128 packed rows, two per CTA when the group fills them.
@@ -238,6 +245,7 @@ fp2_status validate(const fp2_problem* p, const fp2_sparse_params* s, Ctx& c) {
   c.off_vbar = o;   o += align_up(w.vbar_bytes);
   c.off_kbm = o;    o += align_up(w.kbar_mma_bytes);
   c.off_vbm = o;    o += align_up(w.vbar_mma_bytes);
+  c.off_v16 = o;    o += align_up(w.v16_bytes);
   c.off_rowptr = o; o += align_up(w.row_ptr_bytes);
   c.off_colidx = o; o += align_up(w.col_idx_bytes);
   w.prefill_scratch_bytes = o;
@@ -271,9 +279,10 @@ fp2_status encode_3d(CUtensorMap* m, fp2_dtype dt, const void* base, int D, int 
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return fail(FP2_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
   const int elt = elt_bytes(dt);
-  const CUtensorMapDataType t = dt == FP2_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                : dt == FP2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapDataType t = dt == FP2_F32       ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dt == FP2_BF16    ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                : dt == kOperandF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                    : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(heads),
                               static_cast<cuuint64_t>(std::max<int64_t>(rows, 1))};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elt, static_cast<cuuint64_t>(row_stride_elems) * elt};
@@ -299,12 +308,14 @@ fp2_status check_scratch(const void* scratch, size_t have, size_t need) {
   return FP2_OK;
 }
 
-fp2_status check_pooled(const fp2_pooled* pl, bool need_q) {
+// need_q: qbar is read or written; need_v16: the E4M3 f16 copy of V is read or written.
+fp2_status check_pooled(const fp2_pooled* pl, bool need_q, bool need_v16) {
   if (pl == nullptr) return fail(FP2_ERR_INVALID_ARG, "pooled is NULL");
   if ((need_q && pl->qbar == nullptr) || pl->kbar == nullptr || pl->vbar == nullptr || pl->kbar_mma == nullptr ||
       pl->vbar_mma == nullptr)
     return fail(FP2_ERR_INVALID_ARG, "pooled buffers must not be NULL");
-  const void* bufs[5] = {pl->qbar, pl->kbar, pl->vbar, pl->kbar_mma, pl->vbar_mma};
+  if (need_v16 && pl->v16 == nullptr) return fail(FP2_ERR_INVALID_ARG, "pooled->v16 must not be NULL for E4M3 inputs");
+  const void* bufs[6] = {pl->qbar, pl->kbar, pl->vbar, pl->kbar_mma, pl->vbar_mma, need_v16 ? pl->v16 : nullptr};
   for (const void* q : bufs)
     if (q != nullptr && !aligned16(q)) return fail(FP2_ERR_INVALID_ARG, "pooled buffers must be 16-byte aligned");
   return FP2_OK;
@@ -342,6 +353,7 @@ fp2_status run_pool(const fp2_problem* p, const fp2_sparse_params* s, const Ctx&
   a.vbar = pl->vbar;
   a.kbar_mma = pl->kbar_mma;
   a.vbar_mma = pl->vbar_mma;
+  a.v16 = p->dtype == FP2_E4M3 ? pl->v16 : nullptr;
   a.kv_prefix_pooled = p->kv_prefix_pooled ? 1 : 0;
   a.status = status_ptr(scratch);
   const cudaError_t e = fp2::launch_pool(p->dtype, a, c.plan, st);
@@ -393,12 +405,23 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   if ((st2 = encode_3d(&a.tm_k, p->dtype, p->k, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box)) != FP2_OK)
     return st2;
   const bool v32 = p->dtype == FP2_F32;
-  if ((st2 = encode_3d(&a.tm_v, p->dtype, p->v, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box, v32)) != FP2_OK)
+  const bool e4 = p->dtype == FP2_E4M3;
+  // E4M3: the PV operand is the f16 copy of V written by fp2_pool (contiguous rows in key-token
+  // order even for a paged cache) and the f16 pooled vbar.
+  a.v_contig = e4 ? 1 : 0;
+  if (e4) {
+    if ((st2 = encode_3d(&a.tm_v, kOperandF16, pl->v16, D, p->num_kv_heads, c.Tk,
+                         static_cast<int64_t>(p->num_kv_heads) * D, B)) != FP2_OK)
+      return st2;
+  } else if ((st2 = encode_3d(&a.tm_v, p->dtype, p->v, D, p->num_kv_heads, kv_rows, p->kv_stride_tok, kv_box, v32)) !=
+             FP2_OK) {
     return st2;
+  }
   const int64_t hd = static_cast<int64_t>(p->num_kv_heads) * D;
   if ((st2 = encode_3d(&a.tm_kb, p->dtype, pl->kbar_mma, D, p->num_kv_heads, c.total_k_blocks, hd, B)) != FP2_OK)
     return st2;
-  if ((st2 = encode_3d(&a.tm_vb, p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_k_blocks, hd, B, v32)) != FP2_OK)
+  if ((st2 = encode_3d(&a.tm_vb, e4 ? kOperandF16 : p->dtype, pl->vbar_mma, D, p->num_kv_heads, c.total_k_blocks, hd,
+                       B, v32)) != FP2_OK)
     return st2;
   // Output tiles of full blocks go out through TMA stores (16-byte aligned output, no KV split);
   // everything else through per-thread stores.
@@ -506,7 +529,7 @@ fp2_status discover_fixed_scratch(const fp2_problem* problem, const fp2_sparse_p
     return fail(FP2_ERR_UNSUPPORTED, "problem needs " + std::to_string(c.ws.discover_scratch_bytes) +
                                          " bytes of discovery scratch; the static buffer holds " +
                                          std::to_string(capacity));
-  if ((s = check_pooled(pooled, true)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, true, false)) != FP2_OK) return s;
   if ((s = check_index(index, c)) != FP2_OK) return s;
   if ((s = clear_status(scratch, st)) != FP2_OK) return s;
   if (c.T > 0 && (s = run_discover(problem, params, c, pooled, index, scratch, st)) != FP2_OK) return s;
@@ -539,7 +562,7 @@ fp2_status fp2_workspace_size(const fp2_problem* problem, const fp2_sparse_param
   const fp2_workspace& w = c.ws;
   if (pooled_bytes != nullptr)
     *pooled_bytes = align_up(w.qbar_bytes) + align_up(w.kbar_bytes) + align_up(w.vbar_bytes) +
-                    align_up(w.kbar_mma_bytes) + align_up(w.vbar_mma_bytes);
+                    align_up(w.kbar_mma_bytes) + align_up(w.vbar_mma_bytes) + align_up(w.v16_bytes);
   if (index_bytes != nullptr) *index_bytes = align_up(w.row_ptr_bytes) + align_up(w.col_idx_bytes);
   if (scratch_bytes != nullptr) *scratch_bytes = w.scratch_bytes;
   g_last_error.clear();
@@ -552,7 +575,7 @@ fp2_status fp2_pool(const fp2_problem* problem, const fp2_sparse_params* params,
   fp2_status s;
   if ((s = validate(problem, params, c)) != FP2_OK) return s;
   if ((s = check_scratch(scratch, scratch_bytes, c.ws.scratch_bytes)) != FP2_OK) return s;
-  if ((s = check_pooled(pooled, true)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, true, problem->dtype == FP2_E4M3)) != FP2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = clear_status(scratch, st)) != FP2_OK) return s;
   if (c.T == 0) return FP2_OK;
@@ -565,7 +588,7 @@ fp2_status fp2_discover(const fp2_problem* problem, const fp2_sparse_params* par
   fp2_status s;
   if ((s = validate(problem, params, c)) != FP2_OK) return s;
   if ((s = check_scratch(scratch, scratch_bytes, c.ws.scratch_bytes)) != FP2_OK) return s;
-  if ((s = check_pooled(pooled, true)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, true, false)) != FP2_OK) return s;
   if ((s = check_index(index, c)) != FP2_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = clear_status(scratch, st)) != FP2_OK) return s;
@@ -580,7 +603,7 @@ fp2_status fp2_attend(const fp2_problem* problem, const fp2_sparse_params* param
   fp2_status s;
   if ((s = validate(problem, params, c)) != FP2_OK) return s;
   if ((s = check_scratch(scratch, scratch_bytes, c.ws.scratch_bytes)) != FP2_OK) return s;
-  if ((s = check_pooled(pooled, false)) != FP2_OK) return s;
+  if ((s = check_pooled(pooled, false, problem->dtype == FP2_E4M3)) != FP2_OK) return s;
   if ((s = check_index(index, c)) != FP2_OK) return s;
   if (out == nullptr || !aligned16(out)) return fail(FP2_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -598,7 +621,8 @@ fp2_status fp2_prefill(const fp2_problem* problem, const fp2_sparse_params* para
   if (out == nullptr || !aligned16(out)) return fail(FP2_ERR_INVALID_ARG, "out must be a 16-byte aligned pointer");
   char* base = static_cast<char*>(scratch);
   fp2_pooled pl{reinterpret_cast<float*>(base + c.off_qbar), reinterpret_cast<float*>(base + c.off_kbar),
-                reinterpret_cast<float*>(base + c.off_vbar), base + c.off_kbm, base + c.off_vbm};
+                reinterpret_cast<float*>(base + c.off_vbar), base + c.off_kbm, base + c.off_vbm,
+                c.ws.v16_bytes ? base + c.off_v16 : nullptr};
   fp2_index ix{reinterpret_cast<int32_t*>(base + c.off_rowptr), reinterpret_cast<int32_t*>(base + c.off_colidx),
                std::max<int64_t>(c.cap, 1)};
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -23,6 +23,7 @@ struct PoolArgs {
   float* vbar;
   void* kbar_mma;
   void* vbar_mma;
+  void* v16;             // E4M3: f16 copy of V in key-token order (NULL otherwise)
   int kv_prefix_pooled;  // skip K/V of prefix blocks (already pooled)
   uint32_t* status;
 };
@@ -45,11 +46,12 @@ struct DiscArgs {
 struct AttnArgs {
   CUtensorMap tm_q;   // Q  [T, Hq, d]       box {128B / elt, 1, B}
   CUtensorMap tm_k;   // K  tokens (flat)    box {128B / elt, 1, B or page rows}
-  CUtensorMap tm_v;
+  CUtensorMap tm_v;   // V, or for E4M3 inputs its f16 copy [Tk, Hkv, d] (contiguous, box {64, 1, B})
   CUtensorMap tm_kb;  // kbar_mma [blocks, Hkv, d] box {128B / elt, 1, B}
   CUtensorMap tm_vb;
   CUtensorMap tm_o;   // out [T, Hq, d] (bf16, or f32 for f32 inputs) box {128B / elt, 1, B}
   int o_tma;          // 1: full blocks are written through tm_o by TMA stores
+  int v_contig;       // 1: V tiles come from tm_v's contiguous rows even when K is paged (E4M3)
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const int32_t* page_table;  // NULL -> contiguous

@@ -140,6 +140,32 @@ __global__ void __launch_bounds__(128) pool_kernel(const __grid_constant__ PoolA
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       if (t + u < n) accumulate<DT>(buf[u], acc);
+    if constexpr (DT == 2) {
+      // E4M3: the V rows are also written as f16 (exact), in key-token order, for the f16 PV
+      // product of the attention kernel.
+      if (which == 2) {
+        uint16_t* v16 = static_cast<uint16_t*>(a.v16);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (t + u < n) {
+            const int64_t trow = static_cast<int64_t>(P.k_tok_off[r]) + t0 + t + u;
+            const uint32_t w[4] = {buf[u].x, buf[u].y, buf[u].z, buf[u].w};
+            uint4 h0, h1;
+            h0.x = e4m3x2_to_f16x2(w[0] & 0xFFFFu);
+            h0.y = e4m3x2_to_f16x2(w[0] >> 16);
+            h0.z = e4m3x2_to_f16x2(w[1] & 0xFFFFu);
+            h0.w = e4m3x2_to_f16x2(w[1] >> 16);
+            h1.x = e4m3x2_to_f16x2(w[2] & 0xFFFFu);
+            h1.y = e4m3x2_to_f16x2(w[2] >> 16);
+            h1.z = e4m3x2_to_f16x2(w[3] & 0xFFFFu);
+            h1.w = e4m3x2_to_f16x2(w[3] >> 16);
+            uint4* dst16 = reinterpret_cast<uint4*>(v16 + trow * a.Hkv * a.D + col);
+            dst16[0] = h0;
+            dst16[1] = h1;
+          }
+        }
+      }
+    }
   }
 
   const float descale = which == 0 ? a.q_descale : (which == 1 ? a.k_descale : a.v_descale);
@@ -156,7 +182,16 @@ __global__ void __launch_bounds__(128) pool_kernel(const __grid_constant__ PoolA
     d4[e] = make_float4(mean_raw[4 * e] * descale, mean_raw[4 * e + 1] * descale, mean_raw[4 * e + 2] * descale,
                         mean_raw[4 * e + 3] * descale);
 
-  if (which != 0) {
+  if (DT == 2 && which == 2) {
+    // E4M3 vbar operand: f16 (the PV product runs in f16), stored-value domain.
+    uint4 h[2];
+    uint32_t* hw = reinterpret_cast<uint32_t*>(h);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) hw[e] = pack_f16x2(mean_raw[2 * e], mean_raw[2 * e + 1]);
+    uint4* d16 = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.vbar_mma) + static_cast<int64_t>(out_row) * H * a.D + col);
+    d16[0] = h[0];
+    d16[1] = h[1];
+  } else if (which != 0) {
     // Narrow copy in the MMA operand type (E4M3 stays in the stored, un-descaled domain).
     char* nb = static_cast<char*>(which == 1 ? a.kbar_mma : a.vbar_mma);
     uint4 out;

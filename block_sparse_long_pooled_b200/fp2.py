@@ -59,7 +59,7 @@ class fp2_sparse_params(ctypes.Structure):
 
 class fp2_pooled(ctypes.Structure):
     _fields_ = [("qbar", ctypes.c_void_p), ("kbar", ctypes.c_void_p), ("vbar", ctypes.c_void_p),
-                ("kbar_mma", ctypes.c_void_p), ("vbar_mma", ctypes.c_void_p)]
+                ("kbar_mma", ctypes.c_void_p), ("vbar_mma", ctypes.c_void_p), ("v16", ctypes.c_void_p)]
 
 
 class fp2_index(ctypes.Structure):
@@ -74,7 +74,7 @@ class fp2_workspace(ctypes.Structure):
         ("kbar_mma_bytes", ctypes.c_size_t), ("vbar_mma_bytes", ctypes.c_size_t),
         ("row_ptr_bytes", ctypes.c_size_t), ("col_idx_bytes", ctypes.c_size_t),
         ("discover_scratch_bytes", ctypes.c_size_t), ("scratch_bytes", ctypes.c_size_t),
-        ("prefill_scratch_bytes", ctypes.c_size_t),
+        ("prefill_scratch_bytes", ctypes.c_size_t), ("v16_bytes", ctypes.c_size_t),
     ]
 
 
@@ -272,15 +272,23 @@ def alloc_pooled(ws: fp2_workspace, problem: Problem, device):
     s = problem.struct
     nq, nk, Hq, Hkv, D = ws.total_q_blocks, ws.total_kv_blocks, s.num_q_heads, s.num_kv_heads, s.head_dim
     mma_dtype = {FP2_F32: torch.float32, FP2_BF16: torch.bfloat16, FP2_E4M3: torch.uint8}[s.dtype]
+    # the V side of the PV product is f16 for E4M3 inputs (pooled vbar and the copy of V)
+    v_dtype = torch.float16 if s.dtype == FP2_E4M3 else mma_dtype
     t = {
         "qbar": torch.empty((nq, Hq, D), dtype=torch.float32, device=device),
         "kbar": torch.empty((nk, Hkv, D), dtype=torch.float32, device=device),
         "vbar": torch.empty((nk, Hkv, D), dtype=torch.float32, device=device),
         "kbar_mma": torch.empty((nk, Hkv, D), dtype=mma_dtype, device=device),
-        "vbar_mma": torch.empty((nk, Hkv, D), dtype=mma_dtype, device=device),
+        "vbar_mma": torch.empty((nk, Hkv, D), dtype=v_dtype, device=device),
     }
-    st = fp2_pooled(*(_ptr(t[k]) for k in ("qbar", "kbar", "vbar", "kbar_mma", "vbar_mma")))
-    return st, t
+    if s.dtype == FP2_E4M3:
+        t["v16"] = torch.empty((ws.total_kv_tokens, Hkv, D), dtype=torch.float16, device=device)
+    return pooled_struct(t), t
+
+
+def pooled_struct(t: dict) -> fp2_pooled:
+    """fp2_pooled from a dict of tensors (qbar, kbar, vbar, kbar_mma, vbar_mma and, for E4M3, v16)."""
+    return fp2_pooled(*(_ptr(t.get(k)) for k in ("qbar", "kbar", "vbar", "kbar_mma", "vbar_mma", "v16")))
 
 
 def index_struct(row_ptr, col_idx) -> fp2_index:

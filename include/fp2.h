@@ -143,14 +143,20 @@ typedef struct {
                                beyond that stay whole.  Range >= -FP2_MAX_BLOCKS. */
 } fp2_sparse_params;
 
-/* Pooled block statistics (caller-owned device buffers). */
+/* Pooled block statistics and operand copies (caller-owned device buffers, written by fp2_pool). */
 typedef struct {
   float* qbar;     /* [total_q_blocks, Hq, d] f32 block means of Q (dequantised) */
   float* kbar;     /* [total_kv_blocks, Hkv, d] f32 */
   float* vbar;     /* [total_kv_blocks, Hkv, d] f32 */
   void* kbar_mma;  /* [total_kv_blocks, Hkv, d] in dtype: the kbar operand of the correction MMA
                       (E4M3: mean of the stored values, rounded to e4m3, same descale as K) */
-  void* vbar_mma;  /* [total_kv_blocks, Hkv, d] in dtype, likewise for V */
+  void* vbar_mma;  /* [total_kv_blocks, Hkv, d] in the PV operand type: dtype for F32 and BF16, f16 for
+                      E4M3 (mean of the stored values rounded to f16, same descale as V) */
+  void* v16;       /* E4M3 only: [total_kv_tokens, Hkv, d] f16, the stored V values converted exactly
+                      (every e4m3 value is an f16 value), rows in key-token order of cu_seqlens_k
+                      (gathered from the page table when paged); the PV operand of fp2_attend.  With
+                      kv_prefix_pooled the prefix rows must already be there, like kbar/vbar.  NULL
+                      (and unused) for F32 and BF16. */
 } fp2_pooled;
 
 /* CSR index of kept key blocks: row = (q_block_offset_r + i) * Hkv + g for query block i of
@@ -175,6 +181,7 @@ typedef struct {
   size_t scratch_bytes;          /* scratch for fp2_pool / fp2_discover / fp2_attend (adds KV-split partials:
                                     for adaptive splits up to 768 ranges x (128 or 256) rows x d fp32) */
   size_t prefill_scratch_bytes;  /* scratch for fp2_prefill (adds pooled and index buffers) */
+  size_t v16_bytes;              /* fp2_pooled.v16 (E4M3; 0 otherwise) */
 } fp2_workspace;
 
 /* Validate a problem and report buffer sizes.  Host only; launches nothing. */
@@ -182,14 +189,16 @@ FP2_API fp2_status fp2_workspace_query(const fp2_problem* problem, const fp2_spa
                                fp2_workspace* out);
 
 /* The same validation, reporting three totals for callers that carve buffers out of single
- * allocations: pooled_bytes holds the five fp2_pooled buffers and index_bytes row_ptr and col_idx,
+ * allocations: pooled_bytes holds the fp2_pooled buffers (five, plus v16 for E4M3) and index_bytes
+ * row_ptr and col_idx,
  * each buffer starting at a 256-byte aligned offset in that order; scratch_bytes is
  * fp2_workspace.scratch_bytes.  Any output pointer may be NULL.  Host only; launches nothing. */
 FP2_API fp2_status fp2_workspace_size(const fp2_problem* problem, const fp2_sparse_params* params,
                               size_t* pooled_bytes, size_t* index_bytes, size_t* scratch_bytes);
 
 /* Stage 1a (Figure 3, "pools block-mean statistics"): one pass over Q, K, V
- * (gathered through the page table when paged) writing every field of *pooled.
+ * (gathered through the page table when paged) writing every field of *pooled
+ * (for E4M3 also the f16 copy of V that fp2_attend reads).
  * Clears the device status word at the start of scratch. */
 FP2_API fp2_status fp2_pool(const fp2_problem* problem, const fp2_sparse_params* params, const fp2_pooled* pooled,
                     void* scratch, size_t scratch_bytes, fp2_stream_t stream);
@@ -204,7 +213,8 @@ FP2_API fp2_status fp2_discover(const fp2_problem* problem, const fp2_sparse_par
  * with mean correction for the pruned ones.  out: [T, Hq, d] bf16 (f32 when dtype
  * is FP2_F32); lse: [Hq, T] f32 natural-log normaliser, or NULL.  The index may
  * come from fp2_discover or from the caller; every row must be ascending, within
- * [0, i] and contain the diagonal block i. */
+ * [0, i] and contain the diagonal block i.  E4M3: QK runs on the e4m3 Q and K, PV on
+ * the f16 copy of V in pooled->v16 (so fp2_pool must have run on the same problem). */
 FP2_API fp2_status fp2_attend(const fp2_problem* problem, const fp2_sparse_params* params, const fp2_pooled* pooled,
                       const fp2_index* index, void* out, float* lse, void* scratch, size_t scratch_bytes,
                       fp2_stream_t stream);

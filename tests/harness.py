@@ -182,10 +182,14 @@ def compare_pooled(run: GpuRun, inp: W.Inputs, ora: list):
         scale = max(1.0, float(np.abs(ov).max()))
         err = float(np.abs(gv - ov).max())
         assert err <= 2e-5 * scale, (name, err, scale)
-    # narrow MMA copies: one rounding of the fp32 mean to the operand type
+    # narrow MMA copies: one rounding of the fp32 mean to the operand type (the V side is f16 for
+    # e4m3 inputs)
     for name, ov, ds in (("kbar_mma", kb, inp.k_descale), ("vbar_mma", vb, inp.v_descale)):
         t = run.pooled[name]
-        if w.dtype == "e4m3":
+        if w.dtype == "e4m3" and name == "vbar_mma":
+            gv = t.float().cpu().numpy().astype(np.float64) * ds
+            tol = np.abs(ov) * 2.0 ** -10 + 2.0 ** -24 * ds + 1e-9
+        elif w.dtype == "e4m3":
             gv = t.view(torch.float8_e4m3fn).float().cpu().numpy().astype(np.float64) * ds
             tol = np.abs(ov) * 2.0 ** -3 + 2.0 ** -9 * ds + 1e-6
         elif w.dtype == "bf16":
@@ -195,6 +199,9 @@ def compare_pooled(run: GpuRun, inp: W.Inputs, ora: list):
             gv = t.cpu().numpy().astype(np.float64)
             tol = np.abs(ov) * 1e-5 + 1e-6
         assert np.all(np.abs(gv - ov) <= tol), name
+    if w.dtype == "e4m3":
+        # the f16 copy of V equals the stored e4m3 values exactly, rows in key-token order
+        assert torch.equal(run.pooled["v16"].cpu(), inp.v.to(torch.float16)), "v16"
 
 
 def gpu_kept(run: GpuRun, inp: W.Inputs) -> list:

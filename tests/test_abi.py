@@ -98,6 +98,22 @@ def test_workspace_size_totals():
                                          ws.vbar_mma_bytes))
     assert index == up(ws.row_ptr_bytes) + up(ws.col_idx_bytes)
     assert scratch == ws.scratch_bytes
+    assert ws.v16_bytes == 0
+
+
+def test_e4m3_v_side_sizes():
+    """E4M3 inputs: kbar_mma stays e4m3, the V side of the PV product (vbar_mma and the copy of V)
+    is f16, and the pooled total includes the copy."""
+    prob = _problem(dtype=torch.float8_e4m3fn, paged=True)
+    params = fp2.make_params(128)
+    ws = fp2.fp2_workspace_query(prob, params)
+    assert ws.kbar_mma_bytes == 11 * 2 * 128 * 1 and ws.vbar_mma_bytes == 11 * 2 * 128 * 2
+    assert ws.v16_bytes == 1333 * 2 * 128 * 2
+    pooled, _, _ = fp2.fp2_workspace_size(prob, params)
+    up = lambda x: (x + 255) // 256 * 256
+    assert pooled == sum(up(b) for b in (ws.qbar_bytes, ws.kbar_bytes, ws.vbar_bytes, ws.kbar_mma_bytes,
+                                         ws.vbar_mma_bytes, ws.v16_bytes))
+    assert ws.prefill_scratch_bytes >= ws.scratch_bytes + ws.v16_bytes
     # every output is optional; validation is the same as fp2_workspace_query's
     lib = fp2.load_library()
     assert lib.fp2_workspace_size(ctypes.byref(prob.struct), ctypes.byref(params), None, None, None) == fp2.FP2_OK

@@ -165,7 +165,7 @@ def test_prefix_pooled_in_an_earlier_call_is_reused():
     # shared kbar/vbar buffers sized for chunk 2; qbar sized for the larger chunk
     _, pooled = fp2.alloc_pooled(ws2, p2, "cuda")
     pooled["qbar"] = torch.empty((ws1.total_q_blocks, 8, 128), dtype=torch.float32, device="cuda")
-    pst = fp2.fp2_pooled(*(pooled[n].data_ptr() for n in ("qbar", "kbar", "vbar", "kbar_mma", "vbar_mma")))
+    pst = fp2.pooled_struct(pooled)
     scratch = fp2.alloc_scratch(max(ws1.prefill_scratch_bytes, ws2.prefill_scratch_bytes), "cuda")
     kv_names = ("kbar", "vbar", "kbar_mma", "vbar_mma")
 
