@@ -45,7 +45,8 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
 # taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
-ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7531338496 + 1064892416, "source_sha": "804a18555d188493"}}
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7527176704 + 1040678656, "source_sha": "364f4857cd7a8750"},
+                "llama8b_128k_e4m3": {"bytes": 5475396608 + 1029719296, "source_sha": "364f4857cd7a8750"}}
 
 
 def max_over_ranks(pg, x, device=None):
@@ -56,6 +57,14 @@ def max_over_ranks(pg, x, device=None):
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     pg.all_reduce(t, op=pg.ReduceOp.MAX)
     return float(t.item())
+
+
+def attention_traffic(wname):
+    """DRAM bytes of one attention launch from the committed ncu capture, or None when the kernel
+    source changed since it was taken (or no capture exists for the workload)."""
+    tr = ATTN_TRAFFIC.get(wname)
+    sha = source_sha(os.path.join(ROOT, "block_sparse_long_pooled_b200", "csrc", "attention.cu"))
+    return tr["bytes"] if tr is not None and tr["source_sha"] == sha else None
 
 
 def whole_job_value(flops_per_rank_step, world, ms_per_step):
@@ -700,7 +709,8 @@ def measure_config(wname, dev, peaks, steps, warmup, all_kept=True, cpu_pairs=0,
          "ms_per_step": ms, "stages_ms": st, "dense_equiv_tflops": dense / (ms * 1e-3) / 1e12,
          "achieved_tflops": ach / (ms * 1e-3) / 1e12, "sparsity": kept / causal,
          "roofline": {"kernel": "attention_kernel", "bound": "tensor", "achieved": attn, "peak": peak,
-                      "unit": "TFLOP/s", "frac": attn / peak, "peak_source": peak_src},
+                      "unit": "TFLOP/s", "frac": attn / peak, "peak_source": peak_src,
+                      "traffic": attention_traffic(wname)},
          "pool_roofline": {"bound": "hbm", "achieved": pool_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                            "frac": pool_gbs / peaks["hbm_gbs"]},
          "discover_roofline": disc_rl, "stage1_roofline": st1_rl,
@@ -788,9 +798,7 @@ def main():
     value = whole_job_value(dense, world, ms)
     attn_tflops = ach / (stages["attend"] * 1e-3) / 1e12
     peak, peak_src = attention_peak(w.dtype, peaks)
-    sha = source_sha(os.path.join(ROOT, "block_sparse_long_pooled_b200", "csrc", "attention.cu"))
-    tr = ATTN_TRAFFIC.get(w.name)
-    traffic = tr["bytes"] if tr is not None and tr["source_sha"] == sha else None
+    traffic = attention_traffic(w.name)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
