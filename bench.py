@@ -268,6 +268,9 @@ class Path:
         nb = self.ws.total_q_blocks  # q_len == kv_len in the benchmark workloads
         read = T * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * elt
         write = nb * (w.num_q_heads + 2 * w.num_kv_heads) * w.head_dim * 4 + 2 * nb * w.num_kv_heads * w.head_dim * elt
+        if w.dtype == "e4m3":
+            # f16 vbar operand (2 bytes instead of 1) and the f16 copy of V
+            write += nb * w.num_kv_heads * w.head_dim + T * w.num_kv_heads * w.head_dim * 2
         return read + write
 
 
@@ -843,7 +846,7 @@ def main():
                     per.append({"label": label, "workload": wname, "same_as": "headline line"})
                     continue
                 per.append(measure_config(wname, dev, peaks, max(5, args.steps // 2), args.warmup,
-                                          cpu_pairs=48 if rank == 0 else 0, label=label))
+                                          cpu_pairs=128 if rank == 0 else 0, label=label))
             line["per_config"] = per
             fp8 = next(e for e in per if e["workload"] == FP8_WORKLOAD)
             line["fp8"] = {"workload": FP8_WORKLOAD, "ms_per_step": fp8["ms_per_step"],
