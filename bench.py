@@ -829,9 +829,9 @@ def main():
                             "attend_tflops": dach / (dst["attend"] * 1e-3) / 1e12,
                             "attend_frac": dach / (dst["attend"] * 1e-3) / 1e12 / peak}
         del dense_path
-        # at least 16 pipelined steps, so the fill (first upload) and drain (last compute and
+        # at least 32 pipelined steps, so the fill (first upload) and drain (last compute and
         # download) weigh little against the upload-bound steady state
-        e2e_ms, serial_ms, h2d, d2h = time_e2e(path, max(16, args.steps // 2))
+        e2e_ms, serial_ms, h2d, d2h = time_e2e(path, max(32, args.steps))
         e2e_ms = max_over_ranks(pg, e2e_ms, dev)
         line["e2e"] = {"value": whole_job_value(dense, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -192,3 +192,48 @@ def test_prefix_pooled_in_an_earlier_call_is_reused():
     fp2.fp2_pool(p2_reuse, params, pst, scratch)
     torch.cuda.synchronize()
     assert bool((pooled["kbar"][:8] == 7.0).all()) and not bool((pooled["kbar"][8:] == 7.0).any())
+
+
+def test_prefix_pooled_reuse_e4m3_keeps_the_v_copy():
+    """E4M3 chunked prefill with kv_prefix_pooled: the prefix rows of the f16 copy of V (read by the
+    PV product) come from the earlier chunk's fp2_pool, like kbar/vbar, and the result equals a
+    fresh pooling of the whole key range; paged K/V, 64-token pages."""
+    from block_sparse_long_pooled_b200 import fp2
+    w = W.Workload(name="chunk_reuse_e4m3", seqlens=(1500,), num_q_heads=8, num_kv_heads=2, head_dim=128,
+                   block_size=128, dtype="e4m3", sink_blocks=1, window_blocks=2, alpha=0.1, seed=29,
+                   paged=True, page_size=64)
+    inp = W.generate(w)
+    params = Hn.gpu_params(w)
+    dev = Hn.to_device(inp)
+    kc, vc, pt = dev["k_cache"], dev["v_cache"], dev["page_table"]
+    q1, q2 = dev["q"][:1024], dev["q"][1024:]
+    ds = (inp.q_descale, inp.k_descale, inp.v_descale)
+    p1 = fp2.make_problem(q1, kc, vc, [0, 1024], 2, *ds, page_table=pt, cu_seqlens_k=[0, 1024])
+    p2 = fp2.make_problem(q2, kc, vc, [0, 476], 2, *ds, page_table=pt, cu_seqlens_k=[0, 1500])
+    p2_reuse = fp2.make_problem(q2, kc, vc, [0, 476], 2, *ds, page_table=pt, cu_seqlens_k=[0, 1500],
+                                kv_prefix_pooled=True)
+    ws1, ws2 = fp2.fp2_workspace_query(p1, params), fp2.fp2_workspace_query(p2, params)
+    _, pooled = fp2.alloc_pooled(ws2, p2, "cuda")
+    pooled["qbar"] = torch.empty((ws1.total_q_blocks, 8, 128), dtype=torch.float32, device="cuda")
+    pst = fp2.pooled_struct(pooled)
+    scratch = fp2.alloc_scratch(max(ws1.prefill_scratch_bytes, ws2.prefill_scratch_bytes), "cuda")
+
+    def chunk2(prob):
+        fp2.fp2_pool(prob, params, pst, scratch)
+        ist, _ = fp2.alloc_index(ws2, "cuda")
+        fp2.fp2_discover(prob, params, pst, ist, scratch)
+        out = torch.empty(q2.shape, dtype=torch.bfloat16, device="cuda")
+        fp2.fp2_attend(prob, params, pst, ist, out, None, scratch)
+        torch.cuda.synchronize()
+        assert fp2.fp2_get_device_status(scratch) == (0, 0)
+        return out
+
+    for n in ("kbar", "vbar", "kbar_mma", "vbar_mma", "v16"):
+        pooled[n].zero_()
+    fresh = chunk2(p2)
+    for n in ("kbar", "vbar", "kbar_mma", "vbar_mma", "v16"):
+        pooled[n].zero_()
+    fp2.fp2_pool(p1, params, pst, scratch)   # chunk 1 pools key blocks 0-7 and V rows 0-1023
+    reused = chunk2(p2_reuse)                # pools key blocks 8-11 and V rows 1024-1499 only
+    assert torch.equal(fresh, reused)
+    assert torch.equal(pooled["v16"].cpu(), inp.v.to(torch.float16))
