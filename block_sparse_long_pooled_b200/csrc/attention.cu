@@ -33,12 +33,16 @@
 //                    an NSLOT ring of shared-memory slots; finally prefetches into L2 the Q tiles
 //                    of the CTA one wave ahead.
 //   warp 9           QK issuer: S = Q_s K^T (SS form) into the shared S buffer.
-//   warp 10          PV issuer: O_s += P_s V (A operand P_s read from TMEM).  The two products
-//                    touch disjoint TMEM, so each is issued the moment its own inputs are ready
-//                    and the tensor pipe interleaves them; one issuer would stall the pipe at
-//                    every wait between groups.  Both issue tcgen05.mma from lane 0 and signal
-//                    mbarriers with tcgen05.commit.
-//   warp 11          idle (it completes warpgroup 2 for the register split).
+//   warps 10, 11     PV issuers for M tiles 0 and 1: O_s += P_s V (A operand P_s read from TMEM).
+//                    The products touch disjoint TMEM, so each is issued the moment its own
+//                    inputs are ready and the tensor pipe interleaves them; one issuer would stall
+//                    the pipe at every wait between groups.  An issuing warp delays the softmax
+//                    warps of its SMSP (clock64 stamps: the quarter on the QK issuer's SMSP ends a
+//                    tile ~800 cycles after the others), and one PV issuer per M tile on two more
+//                    SMSPs measured fastest; giving each QK group its own warp as well was slower.
+//                    All issue tcgen05.mma from lane 0 and signal mbarriers with tcgen05.commit.
+//                    With one M tile warp 11 idles (it completes warpgroup 2 for the register
+//                    split).
 // e4m3 inputs: QK runs on the e4m3 Q and K tiles; V tiles come from the exact f16 copy of V that
 // the pooling pass writes (and the mean-correction vbar tiles from its f16 means), so PV is an f16
 // product with P written as f16.  Converting V here instead would redo it for every row that keeps
@@ -80,7 +84,9 @@ struct AttnCfg {
   static constexpr int KV_BYTES = K_BYTES > V_BYTES ? K_BYTES : V_BYTES;  // ring slot
   static constexpr int TILE_BUDGET = 200 * 1024;
   static constexpr int NSLOT_RAW = (TILE_BUDGET - 2 * Q_BYTES) / KV_BYTES;
-  static constexpr int NSLOT = NSLOT_RAW > 8 ? 8 : NSLOT_RAW;
+  // Even, so that V loads (odd load indices) always land in odd slots: a V slot is released by
+  // the PV products of both M tiles, issued from two warps.
+  static constexpr int NSLOT = (NSLOT_RAW > 8 ? 8 : NSLOT_RAW) & ~1;
   // PV operand type: f16 for e4m3 inputs, else the input type; K extent of one PV MMA.
   static constexpr int PV_KIND = V16 ? 1 : KIND;
   static constexpr uint32_t PV_FMT = V16 ? 0u : FMT;  // kind::f16 format 0 = f16
@@ -106,7 +112,7 @@ struct AttnCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NSLOT * KV_BYTES;
-  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 1 + 2 + 2;
+  static constexpr int NBAR = 2 + 2 * NSLOT + 2 + 2 + 2 + 2 + 2 + 2 + 2 + 2;
   // Output staging for TMA stores: tile s's normalised O (128 rows x d, output type) goes into
   // the shared memory of its own Q tile, free once the tile's last QK product is done; only when
   // it fits there (bf16 and f32 inputs; e4m3 Q tiles are half the size of a bf16 O tile).
@@ -208,8 +214,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* mask_ready = o_done + 2;
   uint64_t* mma_done = mask_ready + 1;
   uint64_t* s_free = mma_done + 1;  // [2]: the S buffer has been copied out by softmax s
-  uint64_t* pv_done = s_free + 2;   // the PV issuer's final commit
-  uint64_t* o_staged = pv_done + 1; // [2]: every row of tile s is staged for the TMA store
+  uint64_t* pv_done = s_free + 2;   // [2]: PV issuer s's final commit
+  uint64_t* o_staged = pv_done + 2; // [2]: every row of tile s is staged for the TMA store
   uint64_t* o_merge = o_staged + 2;    // [2]: piece CTAs: the tile's merge decision is in merge_flag
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -274,11 +280,13 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int k = 0; k < C::NSLOT; ++k) {
       mbar_init(&kv_full[k], 1);
-      mbar_init(&kv_empty[k], 1);
+      // a V slot (odd) is released by both PV issuers when there are two M tiles
+      mbar_init(&kv_empty[k], ((k & 1) && a.NT == 2) ? 2 : 1);
     }
     mbar_init(mask_ready, 1);
     mbar_init(mma_done, 1);
-    mbar_init(pv_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -429,11 +437,11 @@ __global__ void __launch_bounds__(384, 1)
         for (int s = 0; s < a.NT; ++s) mbar_wait_drain(&q_full[s], 0, a.status, a.wait_limit_ns / 5);
         for (int q = max(0, p - C::NSLOT); q < p; ++q) mbar_wait_drain(&kv_full[q % C::NSLOT], (q / C::NSLOT) & 1, a.status, a.wait_limit_ns / 5);
       }
-    } else if (warp == 9 || warp == 10) {
+    } else if (warp == 9 || warp == 10 || (warp == 11 && a.NT == 2)) {
       // ---------------------------------------------------------------- MMA issuers
       // QK issuer (warp 9), for key tile j with NT = 2: QK1(j) once softmax 0 has copied S0(j)
       // out, then QK0(j+1) once softmax 1 has copied S1(j) out; NT = 1: QK0(j+1) after S0(j).
-      // PV issuer (warp 10): PV0(j) once P0(j) is written, then PV1(j).
+      // PV issuers (warp 10 for M tile 0, warp 11 for M tile 1): PV_s(j) once P_s(j) is written.
       // Each warp runs its loop with warp-uniform control flow (every wait is voted) and lane 0
       // issues each tcgen05 instruction (the *_warp wrappers).
       {
@@ -508,20 +516,19 @@ __global__ void __launch_bounds__(384, 1)
             }
             umma_commit_warp(&o_done[s]);
           };
+          // Warp 10 issues tile 0's products, warp 11 tile 1's: the two PV groups of a key tile
+          // come from two warps on two SMSPs (an issuing warp slows the softmax warps of its SMSP).
+          const int s = warp - 10;
           for (int jt = 0; jt < n_local && ok; ++jt) {
             const int qv = 2 * jt + 1;
             if (!(ok = kv_wait(qv))) break;
-            const uint32_t vaddr = slot_addr(qv);
-            for (int s = 0; s < a.NT; ++s) {
-              if (!(ok = wait_all(&p_full[s], jt & 1))) break;
-              tc_fence_after();
-              issue_pv(s, vaddr, jt);
-            }
-            if (!ok) break;
-            umma_commit_warp(&kv_empty[slot_of(qv)]);  // V(jt) fully consumed
+            if (!(ok = wait_all(&p_full[s], jt & 1))) break;
+            tc_fence_after();
+            issue_pv(s, slot_addr(qv), jt);
+            umma_commit_warp(&kv_empty[slot_of(qv)]);  // this tile's share of V(jt) consumed
           }
-          umma_commit_warp(pv_done);
-          if (lane == 0) mbar_wait_drain(pv_done, 0, a.status, a.wait_limit_ns / 5);
+          umma_commit_warp(&pv_done[s]);
+          if (lane == 0) mbar_wait_drain(&pv_done[s], 0, a.status, a.wait_limit_ns / 5);
           __syncwarp();
         }
       }
