@@ -123,12 +123,15 @@ struct AttnCfg {
   static constexpr bool TMA_OUT = O_STAGE_BYTES <= Q_BYTES;
   static constexpr int OFF_MISC = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;
   static constexpr int OFF_MASK = OFF_MISC + 16;
+  // Checked builds: hand-off counters (QK issues, S releases, P writes, PV issues per tile; loads
+  // per ring slot), 16 words.
+  static constexpr int OFF_CHK = OFF_MASK + FP2_MAX_BLOCKS / 8;
   // At least 116 KB so that a second CTA never shares the SM (each CTA holds all 512 TMEM columns).
-  static constexpr int SMEM_RAW = OFF_MASK + FP2_MAX_BLOCKS / 8 + 1024;
+  static constexpr int SMEM_RAW = OFF_CHK + 64 + 1024;
   static constexpr int SMEM_BYTES = SMEM_RAW > 116 * 1024 ? SMEM_RAW : 116 * 1024;
   static_assert(NSLOT >= 4, "K/V ring needs at least four slots (two key tiles in flight)");
   static_assert(O_COL1 + D <= TMEM_COLS, "TMEM budget");
-  static_assert(OFF_BAR % 8 == 0 && OFF_MASK % 16 == 0, "shared-memory alignment");
+  static_assert(OFF_BAR % 8 == 0 && OFF_MASK % 16 == 0 && OFF_CHK % 16 == 0 && NSLOT <= 8, "shared-memory layout");
   static_assert(D % KCH == 0 && BN % UK == 0 && D % 32 == 0 && BN % 32 == 0, "tile shape");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -221,6 +224,19 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* merge_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);  // [2]
   uint32_t* kmask = reinterpret_cast<uint32_t*>(smem + C::OFF_MASK);
+  // Checked builds: chk[s] QK_s issues, chk[2 + s] S releases by softmax s, chk[4 + s] P_s writes,
+  // chk[6 + s] PV_s issues, chk[8 + k] loads into ring slot k.  Each is bumped by the signalling
+  // thread before its arrive or commit; each waiter checks the exact count its own progress implies.
+  volatile uint32_t* chk = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_CHK);
+  auto bump = [&](int k) {
+    if constexpr (FP2_CHECKED != 0) {
+      atomicAdd(const_cast<uint32_t*>(chk + k), 1u);
+      __threadfence_block();
+    }
+  };
+  auto expect = [&](int k, int n) {
+    if constexpr (FP2_CHECKED != 0) fp2_check(chk[k] == static_cast<uint32_t>(n), a.status);
+  };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // CTAs [0, a.adapt) run the planned pieces of long rows (adaptive splits); the rest map to
@@ -288,6 +304,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
     *abort_flag = 0;
+    if constexpr (FP2_CHECKED != 0)
+      for (int k = 0; k < 16; ++k) chk[k] = 0u;
     fence_mbar_init();
   }
   tc_fence_before();
@@ -308,6 +326,7 @@ __global__ void __launch_bounds__(384, 1)
       auto issue_kv = [&](int jt, int j, int q, int kv) {
         if (kv == 0 && (q >> 1) == a.withhold_k_tile) return;  // testing: this load never arrives
         const int slot = q % C::NSLOT;
+        bump(8 + slot);
         // K side in the input type; V side in the PV operand type (f16 for e4m3 inputs).
         const int dch = kv ? C::VDCH : C::DCH, kch = kv ? C::VKCH : C::KCH;
         mbar_arrive_expect_tx(&kv_full[slot], kv ? C::V_BYTES : C::K_BYTES);
@@ -375,7 +394,7 @@ __global__ void __launch_bounds__(384, 1)
         const int prev = e > 0 ? a.col_idx[rs + e - 1] : -1;
         if (j < 0 || j > I || j <= prev)
           bad = true;
-        else
+        else if (fp2_check((j >> 5) < FP2_MAX_BLOCKS / 32, a.status))
           atomicOr(&kmask[j >> 5], 1u << (j & 31));
       }
       if (lane == 0 && a.col_idx[re - 1] != I) bad = true;
@@ -450,7 +469,11 @@ __global__ void __launch_bounds__(384, 1)
         };
         // Loads come in the order K(0), V(0), K(1), V(1), ...: K(j) is load 2j, V(j) load 2j+1.
         auto slot_of = [&](int q) { return q % C::NSLOT; };
-        auto kv_wait = [&](int q) { return wait_all(&kv_full[slot_of(q)], (q / C::NSLOT) & 1); };
+        auto kv_wait = [&](int q) {
+          const bool got = wait_all(&kv_full[slot_of(q)], (q / C::NSLOT) & 1);
+          if (got && lane == 0) expect(8 + slot_of(q), q / C::NSLOT + 1);  // the load of this use
+          return got;
+        };
         auto slot_addr = [&](int q) { return sbase + C::OFF_KV + slot_of(q) * C::KV_BYTES; };
         bool ok = true;
         if (warp == 9) {
@@ -473,6 +496,8 @@ __global__ void __launch_bounds__(384, 1)
                                     bd0 + static_cast<uint64_t>((c * (BN * 128) + koff) >> 4), C::IDESC_S,
                                     k > 0 ? 1u : 0u);
             }
+            if (lane == 0) bump(s);
+            __syncwarp();
             umma_commit_warp(&s_full[s]);
           };
           if (n_local > 0 && ok) {
@@ -487,6 +512,7 @@ __global__ void __launch_bounds__(384, 1)
             const int qk = 2 * jt;
             if (a.NT == 2) {
               if (!wait_all(&s_free[0], jt & 1)) break;  // softmax 0 holds S0(jt)
+              if (lane == 0) expect(2, jt + 1);
               tc_fence_after();
               issue_qk(1, slot_addr(qk));
               umma_commit_warp(&kv_empty[slot_of(qk)]);  // K(jt) fully consumed
@@ -494,6 +520,7 @@ __global__ void __launch_bounds__(384, 1)
             if (jt + 1 < n_local) {
               if (!kv_wait(qk + 2)) break;
               if (!wait_all(&s_free[a.NT - 1], jt & 1)) break;  // the last softmax holds its S(jt)
+              if (lane == 0) expect(2 + a.NT - 1, jt + 1);
               tc_fence_after();
               issue_qk(0, slot_addr(qk + 2));
               if (a.NT == 1) umma_commit_warp(&kv_empty[slot_of(qk + 2)]);
@@ -514,6 +541,8 @@ __global__ void __launch_bounds__(384, 1)
               const uint64_t bd = vd0 + static_cast<uint64_t>((k * C::PV_UK * 128) >> 4);
               umma_ts_warp<C::PV_KIND>(ocol, pcol + k * 8, bd, C::IDESC_PV, (jt > 0 || k > 0) ? 1u : 0u);
             }
+            if (lane == 0) bump(6 + s);
+            __syncwarp();
             umma_commit_warp(&o_done[s]);
           };
           // Warp 10 issues tile 0's products, warp 11 tile 1's: the two PV groups of a key tile
@@ -523,6 +552,7 @@ __global__ void __launch_bounds__(384, 1)
             const int qv = 2 * jt + 1;
             if (!(ok = kv_wait(qv))) break;
             if (!(ok = wait_all(&p_full[s], jt & 1))) break;
+            if (lane == 0) expect(4 + s, jt + 1);
             tc_fence_after();
             issue_pv(s, slot_addr(qv), jt);
             umma_commit_warp(&kv_empty[slot_of(qv)]);  // this tile's share of V(jt) consumed
@@ -542,8 +572,11 @@ __global__ void __launch_bounds__(384, 1)
       constexpr int HS = 128 / BN;
       const int hs = rt / BN, tl = rt % BN;
       const int hl = (part * a.NT + s) * HS + hs;
-      const bool row_ok = (hl < a.G) && (i * BN + tl < L);
+      const bool in_seq = (hl < a.G) && (i * BN + tl < L);
       const int h = g * a.G + min(hl, a.G - 1);
+      // a row of the sequence whose output position lies inside O (the bound is checked in
+      // checked builds)
+      const bool row_ok = in_seq && fp2_check(P.tok_off[r] + i * BN + tl < a.total_tokens && h < a.Hq, a.status);
       const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
       const uint32_t s_addr = tmem + lane_base + C::S_COL;
       const uint32_t p_addr = tmem + lane_base + (s ? C::P_COL1 : C::P_COL0);
@@ -558,6 +591,7 @@ __global__ void __launch_bounds__(384, 1)
         const int jt = t_begin + jl;  // position in the row's key stream
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[s], jl & 1, abort_flag, a.status, a.wait_limit_ns));
         if (!ok) break;
+        if (rt == 0) expect(s, jl + 1);  // QK_s(jl) and nothing later
         tc_fence_after();
         // The whole S row of this thread, in registers.
         uint32_t v[BN];
@@ -566,6 +600,7 @@ __global__ void __launch_bounds__(384, 1)
         else
           tmem_ld64_sync(s_addr, v);
         // S is in registers: hand the buffer to the next QK product.
+        if (rt == 0) bump(2 + s);
         tc_fence_before();
         mbar_arrive(&s_free[s]);
         // PV_s(jl-1) must be complete before O_s is rescaled or P_s is overwritten.
@@ -573,6 +608,7 @@ __global__ void __launch_bounds__(384, 1)
         auto wait_pv_prev = [&]() {
           if (!pv_prev_done) {
             ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (jl - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+            if (ok && rt == 0) expect(6 + s, jl);  // PV_s(jl-1) and nothing later
             tc_fence_after();
             pv_prev_done = true;
           }
@@ -695,6 +731,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         const float rsum = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
         tmem_st_wait();
+        if (rt == 0) bump(4 + s);
         tc_fence_before();
         mbar_arrive(&p_full[s]);
         l_run += rsum;
@@ -702,6 +739,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (ok && done_tiles == n_local && n_local > 0)
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_done[s], (n_local - 1) & 1, abort_flag, a.status, a.wait_limit_ns));
+      if (ok && n_local > 0 && rt == 0) expect(6 + s, n_local);
       tc_fence_after();
       if (item >= 0) {
         // Piece of a split row: its normalised partial O (fp32) and natural-log LSE go to the
@@ -710,6 +748,7 @@ __global__ void __launch_bounds__(384, 1)
         // rows.  No CTA waits for another.  A piece with no visible key contributes LSE = -inf.
         const int prow = a.NT * 128;
         const int64_t srow = static_cast<int64_t>(item) * prow + s * 128 + rt;
+        const bool slot_ok = fp2_check(srow < static_cast<int64_t>(a.adapt) * prow, a.status);  // checked builds
         const bool any = ok && n_local > 0 && l_run > 0.f;
         const float inv = any ? a.v_descale / l_run : 0.f;
         float* op = a.o_slot + srow * D;
@@ -723,12 +762,15 @@ __global__ void __launch_bounds__(384, 1)
             for (int e = 0; e < 32; ++e) v[e] = 0u;
           }
           float4* dst = reinterpret_cast<float4*>(op + c * 32);
+          if (slot_ok) {
   #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
-                                 __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(v[4 * e]) * inv, __uint_as_float(v[4 * e + 1]) * inv,
+                                   __uint_as_float(v[4 * e + 2]) * inv, __uint_as_float(v[4 * e + 3]) * inv);
+          }
         }
-        a.lse_slot[srow] = any ? (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f : -CUDART_INF_F;
+        if (slot_ok)
+          a.lse_slot[srow] = any ? (m_run + log2f(l_run) - C::P_SHIFT) * 0.6931471805599453f : -CUDART_INF_F;
         __threadfence();
         mbar_arrive(&o_staged[s]);
         const int first = item - split;  // first piece of this (row, part)

@@ -640,6 +640,7 @@ fp2_status fp2_get_device_status(const void* scratch, uint32_t* status_out) {
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   *status_out = w;
   if (w & FP2_DEV_TIMEOUT) return fail(FP2_ERR_TIMEOUT, "a device-side wait timed out");
+  if (w & FP2_DEV_CHECK) return fail(FP2_ERR_CHECK_FAILED, "a device-side check of the checked build failed");
   if (w & (FP2_DEV_PAGE_OOB | FP2_DEV_INDEX_OOB | FP2_DEV_CAPACITY))
     return fail(FP2_ERR_DEVICE_BOUNDS, "device reported an out-of-range page id, index entry or capacity overflow");
   return FP2_OK;
@@ -664,5 +665,13 @@ fp2_status fp2_debug_set(int32_t key, int64_t value) {
 const char* fp2_last_error(void) { return g_last_error.c_str(); }
 
 int32_t fp2_version(void) { return 10000; }
+
+uint32_t fp2_build_flags(void) {
+#if defined(FP2_CHECKED) && FP2_CHECKED
+  return FP2_BUILD_CHECKED;
+#else
+  return 0u;
+#endif
+}
 
 }  // extern "C"

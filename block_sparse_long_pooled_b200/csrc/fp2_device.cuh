@@ -25,6 +25,20 @@ FP2_DEVICE uint64_t globaltimer_ns() {
 
 FP2_DEVICE void set_status(uint32_t* status, uint32_t bits) { atomicOr(status, bits); }
 
+// Checked builds (FP2_CHECKED=1): an invariant that does not hold sets FP2_DEV_CHECK and the caller
+// skips the guarded access.  Normal builds compile every check away.
+#ifndef FP2_CHECKED
+#define FP2_CHECKED 0
+#endif
+FP2_DEVICE bool fp2_check(bool cond, uint32_t* status) {
+  if constexpr (FP2_CHECKED != 0) {
+    if (!cond) set_status(status, FP2_DEV_CHECK);
+    return cond;
+  } else {
+    return true;
+  }
+}
+
 // Work item v of a list ordered by level descending (level = query block or query-block tile),
 // `width` items per (sequence, level), sequences with fewer levels dropping out as the level
 // falls.  nlev(r) = ceil(nblk[r] / tile); tile is 1 or P.disc_tile (the two tables the host

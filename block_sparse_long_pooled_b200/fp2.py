@@ -15,19 +15,24 @@ from typing import Optional
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libfp2.so")
+# FP2_LIBRARY selects another build of the same library for this process (the tests use it to
+# run with libfp2_checked.so); by default libfp2.so next to this file.
+LIB_PATH = os.environ.get("FP2_LIBRARY") or os.path.join(_HERE, "libfp2.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libfp2_checked.so")
 
 FP2_OK, FP2_ERR_INVALID_ARG, FP2_ERR_UNSUPPORTED, FP2_ERR_WORKSPACE_TOO_SMALL = 0, 1, 2, 3
-FP2_ERR_CUDA, FP2_ERR_DEVICE_BOUNDS, FP2_ERR_TIMEOUT = 4, 5, 6
+FP2_ERR_CUDA, FP2_ERR_DEVICE_BOUNDS, FP2_ERR_TIMEOUT, FP2_ERR_CHECK_FAILED = 4, 5, 6, 7
 FP2_F32, FP2_BF16, FP2_E4M3 = 0, 1, 2
-FP2_DEV_PAGE_OOB, FP2_DEV_INDEX_OOB, FP2_DEV_CAPACITY, FP2_DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+FP2_DEV_PAGE_OOB, FP2_DEV_INDEX_OOB, FP2_DEV_CAPACITY, FP2_DEV_TIMEOUT, FP2_DEV_CHECK = 0x1, 0x2, 0x4, 0x8, 0x10
+FP2_BUILD_CHECKED = 0x1
 FP2_MAX_SEQS, FP2_MAX_BLOCKS = 512, 4096
 
 STATUS_NAMES = {0: "FP2_OK", 1: "FP2_ERR_INVALID_ARG", 2: "FP2_ERR_UNSUPPORTED", 3: "FP2_ERR_WORKSPACE_TOO_SMALL",
-                4: "FP2_ERR_CUDA", 5: "FP2_ERR_DEVICE_BOUNDS", 6: "FP2_ERR_TIMEOUT"}
+                4: "FP2_ERR_CUDA", 5: "FP2_ERR_DEVICE_BOUNDS", 6: "FP2_ERR_TIMEOUT", 7: "FP2_ERR_CHECK_FAILED"}
 
 EXPORTED = ("fp2_workspace_query", "fp2_workspace_size", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
-            "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static", "fp2_debug_set")
+            "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static", "fp2_debug_set",
+            "fp2_build_flags")
 FP2_DEBUG_WAIT_LIMIT_NS, FP2_DEBUG_WITHHOLD_K_TILE = 1, 2
 FP2_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -114,6 +119,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fp2_last_error.restype = ctypes.c_char_p
     lib.fp2_version.argtypes = []
     lib.fp2_version.restype = ctypes.c_int32
+    lib.fp2_build_flags.argtypes = []
+    lib.fp2_build_flags.restype = ctypes.c_uint32
     _lib = lib
     return lib
 
@@ -262,6 +269,11 @@ def fp2_last_error() -> str:
 
 def fp2_version() -> int:
     return int(load_library().fp2_version())
+
+
+def fp2_build_flags() -> int:
+    """FP2_BUILD_* bits of the loaded library (FP2_BUILD_CHECKED for libfp2_checked.so)."""
+    return int(load_library().fp2_build_flags())
 
 
 # ------------------------------------------------------------------ buffer helpers (torch allocations)

@@ -80,7 +80,8 @@ typedef enum {
   FP2_ERR_WORKSPACE_TOO_SMALL = 3,  /* scratch_bytes below fp2_workspace_query's figure */
   FP2_ERR_CUDA = 4,                 /* a CUDA runtime call failed (message has the CUDA error) */
   FP2_ERR_DEVICE_BOUNDS = 5,        /* device saw a page id / index entry out of range */
-  FP2_ERR_TIMEOUT = 6               /* a device-side wait ran past its time limit */
+  FP2_ERR_TIMEOUT = 6,              /* a device-side wait ran past its time limit */
+  FP2_ERR_CHECK_FAILED = 7          /* checked build: a device-side invariant failed */
 } fp2_status;
 
 typedef enum { FP2_F32 = 0, FP2_BF16 = 1, FP2_E4M3 = 2 } fp2_dtype;
@@ -90,6 +91,8 @@ typedef enum { FP2_F32 = 0, FP2_BF16 = 1, FP2_E4M3 = 2 } fp2_dtype;
 #define FP2_DEV_INDEX_OOB 0x2u     /* CSR column outside [0, i] / not ascending / diagonal missing */
 #define FP2_DEV_CAPACITY 0x4u      /* kept blocks exceed fp2_index.col_capacity */
 #define FP2_DEV_TIMEOUT 0x8u       /* an mbarrier wait gave up */
+#define FP2_DEV_CHECK 0x10u        /* checked build only: a hand-off count or an index bound did not
+                                      hold where it was checked; the guarded access was skipped */
 
 /* cudaStream_t, passed as an opaque pointer so that this header needs no CUDA include. */
 typedef void* fp2_stream_t;
@@ -268,6 +271,16 @@ FP2_API const char* fp2_last_error(void);
 
 /* Library version as major*10000 + minor*100 + patch. */
 FP2_API int32_t fp2_version(void);
+
+/* How this library was built: FP2_BUILD_CHECKED is set in libfp2_checked.so, the same sources
+ * compiled with FP2_CHECKED=1.  There every mbarrier hand-off of the attention kernel is followed
+ * by a check that the producing side has signalled exactly as often as the waiter's own count says
+ * (a wait that completed on a stale or a future phase of the barrier would see a different count),
+ * and per-thread global stores and shared-memory indexes are bounds-checked.  A failed check sets
+ * FP2_DEV_CHECK (fp2_get_device_status returns FP2_ERR_CHECK_FAILED) and skips the guarded store;
+ * nothing traps.  Same arguments and results as the normal library, somewhat slower. */
+#define FP2_BUILD_CHECKED 0x1u
+FP2_API uint32_t fp2_build_flags(void);
 
 #ifdef __cplusplus
 }

@@ -38,6 +38,25 @@ def test_exports_every_declared_symbol():
     assert fp2.fp2_version() == 10000
 
 
+def test_checked_build_exports_the_same_symbols_and_says_so():
+    # libfp2_checked.so: the same sources with FP2_CHECKED=1 (device-side hand-off and bounds checks)
+    B.build(checked=True)
+    decl = declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", B.CHECKED_LIB], capture_output=True, text=True,
+                         check=True).stdout
+    assert sorted(l.split()[-1] for l in out.splitlines() if " T " in l) == decl
+    import ctypes
+    checked = ctypes.CDLL(B.CHECKED_LIB)
+    checked.fp2_build_flags.restype = ctypes.c_uint32
+    assert checked.fp2_build_flags() == fp2.FP2_BUILD_CHECKED
+    if os.environ.get("FP2_LIBRARY") is None:
+        assert fp2.fp2_build_flags() == 0          # the default library has no checks compiled in
+    # the status word's check bit maps to its own error code
+    assert fp2.STATUS_NAMES[fp2.FP2_ERR_CHECK_FAILED] == "FP2_ERR_CHECK_FAILED"
+    assert fp2.FP2_DEV_CHECK not in (fp2.FP2_DEV_PAGE_OOB, fp2.FP2_DEV_INDEX_OOB, fp2.FP2_DEV_CAPACITY,
+                                     fp2.FP2_DEV_TIMEOUT)
+
+
 def _problem(seqlens=(1000, 333), Hq=8, Hkv=2, d=128, dtype=torch.bfloat16, paged=False, page_size=64):
     T = sum(seqlens)
     cu = np.concatenate([[0], np.cumsum(seqlens)]).astype(np.int32)
