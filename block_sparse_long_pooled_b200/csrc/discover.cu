@@ -53,11 +53,13 @@ struct DiscCfg {
   static constexpr int OFF_UNION = (OFF_BAR + NBAR * 8 + 15) / 16 * 16;  // [2][128][4] u32
   static constexpr int OFF_CNT = OFF_UNION + 2 * 128 * 4 * 4;            // [128] int
   static constexpr int OFF_MISC = OFF_CNT + 128 * 4;                     // TMEM address, abort flag
-  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;                // + 1024-byte alignment slack
+  static constexpr int OFF_CHK = OFF_MISC + 16;                          // checked builds: 16 counters
+  static constexpr int SMEM_BYTES = OFF_CHK + 64 + 1024;                 // + 1024-byte alignment slack
   // bf16 x bf16 -> f32, both operands K-major, M = 128, N = 128.
   static constexpr uint32_t IDESC = make_idesc(1u, 1u, 0u, 0u, 128u, 128u);
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-  static_assert(OFF_BAR % 8 == 0 && OFF_UNION % 16 == 0, "shared-memory alignment");
+  static_assert(OFF_BAR % 8 == 0 && OFF_UNION % 16 == 0 && OFF_CHK % 16 == 0 && NST <= 4 && NBUF <= 4,
+                "shared-memory layout");
   static_assert((128 * UPR) % (NCONV * 32) == 0, "converter work split");
 };
 
@@ -153,6 +155,20 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
   int* cnt = reinterpret_cast<int*>(smem + C::OFF_CNT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  // Checked builds: hand-off counters, bumped by the signalling thread before its arrive or commit
+  // and compared by the waiter with the exact count its own progress implies: chk[st] converter
+  // fills of stage st (NCONV per use), chk[4 + st] releases of stage st by the MMA warp, chk[8 + b]
+  // score chunks issued into TMEM buffer b, chk[12 + b] releases of buffer b (4 epilogue warps).
+  volatile uint32_t* chk = reinterpret_cast<volatile uint32_t*>(smem + C::OFF_CHK);
+  auto bump = [&](int k) {
+    if constexpr (FP2_CHECKED != 0) {
+      atomicAdd(const_cast<uint32_t*>(chk + k), 1u);
+      __threadfence_block();
+    }
+  };
+  auto expect = [&](int k, int n) {
+    if constexpr (FP2_CHECKED != 0) fp2_check(chk[k] == static_cast<uint32_t>(n), a.status);
+  };
 
   const int nch = (J1 + C::KEYS - 1) / C::KEYS;
   const int nq = 2 * nch;  // pass 1 then pass 2 over the same chunks
@@ -173,6 +189,8 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
+    if constexpr (FP2_CHECKED != 0)
+      for (int k = 0; k < 16; ++k) chk[k] = 0u;
     fence_mbar_init();
   }
   for (int x = tid; x < 2 * 128 * 4; x += C::THREADS) ubuf[x] = 0u;
@@ -236,9 +254,13 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
       });
       if (use > 0 && !__all_sync(0xFFFFFFFFu, mbar_wait(&b_empty[stage], (use - 1) & 1, abort_flag, a.status)))
         break;
+      if (use > 0 && lane == 0) expect(4 + stage, use);  // the MMA warp released this use's stage
       uint8_t* hb = smem + C::OFF_B + stage * 2 * C::PLANE;
       store(hb, hb + C::PLANE);
-      if (lane == 0) mbar_arrive(&b_full[stage]);
+      if (lane == 0) {
+        bump(stage);
+        mbar_arrive(&b_full[stage]);
+      }
     }
   } else if (warp == 4 + C::NCONV) {
     // ------------------------------------------------------------------ MMA issuer
@@ -246,8 +268,11 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
     for (int q = 0; q < nq && ok; ++q) {
       const int stage = q % C::NST, buf = q % C::NBUF;
       ok = __all_sync(0xFFFFFFFFu, mbar_wait(&b_full[stage], (q / C::NST) & 1, abort_flag, a.status));
-      if (ok && q >= C::NBUF)
+      if (ok && lane == 0) expect(stage, C::NCONV * (q / C::NST + 1));
+      if (ok && q >= C::NBUF) {
         ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_empty[buf], ((q / C::NBUF) - 1) & 1, abort_flag, a.status));
+        if (ok && lane == 0) expect(12 + buf, 4 * (q / C::NBUF));
+      }
       if (!ok) break;
       tc_fence_after();
       const uint32_t dcol = tmem + buf * C::KEYS;
@@ -262,6 +287,11 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
           umma_ss_warp<1>(dcol, ad0 + (off >> 4), bd0 + (off >> 4), C::IDESC, (t > 0 || k > 0) ? 1u : 0u);
         }
       }
+      if (lane == 0) {
+        bump(4 + stage);
+        bump(8 + buf);
+      }
+      __syncwarp();
       umma_commit_warp(&b_empty[stage]);
       umma_commit_warp(&s_full[buf]);
     }
@@ -283,6 +313,7 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
       const int buf = q % C::NBUF, c = q % nch, j0 = c * C::KEYS;
       const bool pass2 = q >= nch;
       if (ok) ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[buf], (q / C::NBUF) & 1, abort_flag, a.status));
+      if (ok && lane == 0) expect(8 + buf, q / C::NBUF + 1);
       if (ok) tc_fence_after();
       if (pass2 && q == nch) thr = mrun + a.ln_alpha;
       const int lim = I - j0;  // columns e <= lim are causal for this row
@@ -294,7 +325,10 @@ __global__ void __launch_bounds__(DiscCfg<D>::THREADS, 1) discover_kernel(const 
         if (hf == 1) {  // the buffer has been read: hand it back to the MMA warp
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&s_empty[buf]);
+          if (lane == 0) {
+            bump(12 + buf);
+            mbar_arrive(&s_empty[buf]);
+          }
         }
         if (!ok || !valid) continue;
         const int lh = lim - hf * 64;  // causal limit within this half
