@@ -45,8 +45,8 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM traffic of one attention launch, from an ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum, one pass) of the same workload; valid only for the kernel source it was
 # taken on (sha256 prefix of csrc/attention.cu), otherwise reported as null.
-ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7548903424 + 1040888064, "source_sha": "e7120442fafbad0c"},
-                "llama8b_128k_e4m3": {"bytes": 5444209920 + 1029414144, "source_sha": "e7120442fafbad0c"}}
+ATTN_TRAFFIC = {"llama8b_128k_bf16": {"bytes": 7598519552 + 1040229120, "source_sha": "e1d1461b29023c2c"},
+                "llama8b_128k_e4m3": {"bytes": 5427795200 + 1029442560, "source_sha": "e1d1461b29023c2c"}}
 
 
 def max_over_ranks(pg, x, device=None):

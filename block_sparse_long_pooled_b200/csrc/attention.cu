@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(384, 1)
         if (kv == 0 && (q >> 1) == a.withhold_k_tile) return;  // testing: this load never arrives
         const int slot = q % C::NSLOT;
         bump(8 + slot);
+        if (q == a.miscount_load) bump(8 + slot);  // testing: a count the consumer does not expect
         // K side in the input type; V side in the PV operand type (f16 for e4m3 inputs).
         const int dch = kv ? C::VDCH : C::DCH, kch = kv ? C::VKCH : C::KCH;
         mbar_arrive_expect_tx(&kv_full[slot], kv ? C::V_BYTES : C::K_BYTES);

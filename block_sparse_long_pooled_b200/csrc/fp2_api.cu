@@ -48,6 +48,7 @@ int elt_bytes(fp2_dtype t) { return t == FP2_F32 ? 4 : ((t == FP2_BF16 || t == k
 // Testing hooks set through fp2_debug_set (process-wide; read when attention launches).
 std::atomic<int64_t> g_wait_limit_ns{0};     // 0: the default limit of 1 s
 std::atomic<int64_t> g_withhold_k_tile{-1};  // -1: every load is issued
+std::atomic<int64_t> g_miscount_load{-1};    // -1: every load is counted once (checked builds)
 
 // Everything derived from (problem, params) on the host.
 struct Ctx {
@@ -466,6 +467,7 @@ fp2_status run_attend(const fp2_problem* p, const fp2_sparse_params* s, const Ct
   const int64_t lim = g_wait_limit_ns.load();
   a.wait_limit_ns = lim > 0 ? static_cast<uint64_t>(lim) : 1000000000ull;
   a.withhold_k_tile = static_cast<int>(g_withhold_k_tile.load());
+  a.miscount_load = static_cast<int>(g_miscount_load.load());
   {
     int dev = 0, nsm = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -656,6 +658,10 @@ fp2_status fp2_debug_set(int32_t key, int64_t value) {
     case FP2_DEBUG_WITHHOLD_K_TILE:
       if (value < -1 || value > FP2_MAX_BLOCKS) return fail(FP2_ERR_INVALID_ARG, "tile must be -1 or in [0, FP2_MAX_BLOCKS]");
       g_withhold_k_tile.store(value);
+      return FP2_OK;
+    case FP2_DEBUG_MISCOUNT_LOAD:
+      if (value < -1 || value > 2 * FP2_MAX_BLOCKS) return fail(FP2_ERR_INVALID_ARG, "load must be -1 or in [0, 2 * FP2_MAX_BLOCKS]");
+      g_miscount_load.store(value);
       return FP2_OK;
     default:
       return fail(FP2_ERR_INVALID_ARG, "unknown debug key");

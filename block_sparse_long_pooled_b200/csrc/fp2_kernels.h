@@ -82,6 +82,7 @@ struct AttnArgs {
   uint32_t* status;
   uint64_t wait_limit_ns;     // limit of every mbarrier wait (drains of in-flight copies: a fifth)
   int withhold_k_tile;        // testing: the producer skips the K load of this local key tile (-1: none)
+  int miscount_load;          // testing, checked builds: the producer counts this load twice (-1: none)
 };
 
 // Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device.  The

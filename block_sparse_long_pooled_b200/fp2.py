@@ -33,7 +33,7 @@ STATUS_NAMES = {0: "FP2_OK", 1: "FP2_ERR_INVALID_ARG", 2: "FP2_ERR_UNSUPPORTED",
 EXPORTED = ("fp2_workspace_query", "fp2_workspace_size", "fp2_pool", "fp2_discover", "fp2_attend", "fp2_prefill",
             "fp2_get_device_status", "fp2_last_error", "fp2_version", "fp2_discover_static", "fp2_debug_set",
             "fp2_build_flags")
-FP2_DEBUG_WAIT_LIMIT_NS, FP2_DEBUG_WITHHOLD_K_TILE = 1, 2
+FP2_DEBUG_WAIT_LIMIT_NS, FP2_DEBUG_WITHHOLD_K_TILE, FP2_DEBUG_MISCOUNT_LOAD = 1, 2, 3
 FP2_STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -259,7 +259,8 @@ def fp2_get_device_status(scratch) -> tuple:
 
 
 def fp2_debug_set(key: int, value: int):
-    """Testing hook (process-wide): FP2_DEBUG_WAIT_LIMIT_NS or FP2_DEBUG_WITHHOLD_K_TILE."""
+    """Testing hook (process-wide): FP2_DEBUG_WAIT_LIMIT_NS, FP2_DEBUG_WITHHOLD_K_TILE or
+    FP2_DEBUG_MISCOUNT_LOAD (checked builds)."""
     _check(load_library().fp2_debug_set(int(key), int(value)))
 
 

@@ -261,9 +261,15 @@ FP2_API fp2_status fp2_discover_static(const fp2_problem* problem, const fp2_spa
  *                              never completes, the wait for it runs out, every role of the CTA
  *                              gives up and drains through its bounded paths, and the status word
  *                              gets FP2_DEV_TIMEOUT.  Nothing faults; the next call is unaffected.
+ *   FP2_DEBUG_MISCOUNT_LOAD    checked builds only: the producer of every attention CTA counts its
+ *                              K/V load `value` (-1 restores normal operation) twice in the
+ *                              hand-off counters, so the consumer's check of that load fails and
+ *                              the status word gets FP2_DEV_CHECK.  The data path is unchanged;
+ *                              the normal build ignores it.
  * Returns FP2_ERR_INVALID_ARG for an unknown key or a value out of range. */
 #define FP2_DEBUG_WAIT_LIMIT_NS 1
 #define FP2_DEBUG_WITHHOLD_K_TILE 2
+#define FP2_DEBUG_MISCOUNT_LOAD 3
 FP2_API fp2_status fp2_debug_set(int32_t key, int64_t value);
 
 /* Message for the last failing call on this thread ("" if none). */

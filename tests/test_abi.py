@@ -226,6 +226,12 @@ def test_debug_hooks_validate_and_reset():
     fp2.fp2_debug_set(fp2.FP2_DEBUG_WAIT_LIMIT_NS, 0)
     fp2.fp2_debug_set(fp2.FP2_DEBUG_WITHHOLD_K_TILE, 3)
     fp2.fp2_debug_set(fp2.FP2_DEBUG_WITHHOLD_K_TILE, -1)
+    with pytest.raises(fp2.FP2Error):
+        fp2.fp2_debug_set(fp2.FP2_DEBUG_MISCOUNT_LOAD, -2)
+    with pytest.raises(fp2.FP2Error):
+        fp2.fp2_debug_set(fp2.FP2_DEBUG_MISCOUNT_LOAD, 2 * fp2.FP2_MAX_BLOCKS + 1)
+    fp2.fp2_debug_set(fp2.FP2_DEBUG_MISCOUNT_LOAD, 2)
+    fp2.fp2_debug_set(fp2.FP2_DEBUG_MISCOUNT_LOAD, -1)
 
 
 def test_sequence_count_limit():
