@@ -47,6 +47,9 @@ CASES = [
     chunk_case("chunk_bf16_varlen_adaptive", (1280, 700, 2000), (256, 700, 720), kv_splits=-2),
     chunk_case("chunk_e4m3_paged_adaptive", (2100, 1500), (564, 220), kv_splits=-3, dtype="e4m3", paged=True,
                page_size=64),
+    # a short chunk after a long prefix (304 prefix + 9 query blocks, 3 key chunks of 128): discovery splits each
+    # tile's key chunks over several CTAs (partial row maxima, then thresholds)
+    chunk_case("chunk_bf16_long_prefix", (40000,), (1088,)),
 ]
 
 
